@@ -1,0 +1,240 @@
+"""CPU oracle of the ragged-bucket 8-bit Adam step (test infrastructure only).
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  It shares no code with the product
+library: the arithmetic lives in ``oracle.cpp`` (plain C++, fp32 in one fixed
+operation order) and this module only marshals numpy arrays.
+
+Every function cites the part of the veScale-FSDP description it follows; the
+parity status of each is stated in ``oracle.cpp``'s header.
+"""
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.cpp")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+OK, EINVAL, EINFEASIBLE = 0, 1, 2
+CXXFLAGS = ["-O2", "-std=c++17", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+            "-fno-fast-math", "-fno-unsafe-math-optimizations"]
+
+
+def build(force=False):
+    """Compile oracle.cpp into liboracle.so (g++, no FMA contraction, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        subprocess.check_call(["g++", *CXXFLAGS, "-o", _LIB, _SRC])
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    build()
+    lib = ctypes.CDLL(_LIB)
+    P = ctypes.c_void_p
+    i32, i64, f32 = ctypes.c_int32, ctypes.c_int64, ctypes.c_float
+    lib.orc_plan.restype = ctypes.c_int
+    lib.orc_plan.argtypes = [P, P, P, i32, i32, i64, i64, i32, P, P]
+    lib.orc_place_fixed.restype = ctypes.c_int
+    lib.orc_place_fixed.argtypes = [P, P, P, i32, i32, i64, i64, i32, P]
+    lib.orc_exists_placement.restype = ctypes.c_int
+    lib.orc_exists_placement.argtypes = [P, P, i32, i64, i32, i64]
+    lib.orc_bruteforce_min_bucket.restype = i64
+    lib.orc_bruteforce_min_bucket.argtypes = [P, P, P, i32, i32, i64]
+    lib.orc_check_layout.restype = ctypes.c_int
+    lib.orc_check_layout.argtypes = [P, P, P, i32, i32, i64, P, i64]
+    lib.orc_adam8_step.restype = None
+    lib.orc_adam8_step.argtypes = [i64, P, P, P, P, P, P, P, P, P, P,
+                                   f32, f32, f32, f32, f32, i64, f32, i32]
+    lib.orc_step_scalars.restype = None
+    lib.orc_step_scalars.argtypes = [f32, f32, f32, f32, f32, i64, P]
+    lib.orc_pack.restype = None
+    lib.orc_pack.argtypes = [i64, P, P, f32]
+    lib.orc_bf16_round.restype = None
+    lib.orc_bf16_round.argtypes = [i64, P, P]
+    _lib = lib
+    return lib
+
+
+def _i64(a):
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int64))
+
+
+def _ptr(a):
+    return a.ctypes.data if a.size else None
+
+
+# ---------------------------------------------------------------- layout ---
+
+def plan(rows, cols, k, m, align=16, max_bucket=0, literal=False):
+    """Structure-aware bucket layout (paper Sec. 4 as the pages give it: sort by
+    block size descending, then place with block alignment at every slice
+    boundary and padding only between tensors).
+
+    Returns (status, offsets[n] in input order, slice size s).
+    """
+    rows, cols, k = _i64(rows), _i64(cols), _i64(k)
+    n = rows.size
+    off = np.zeros(max(n, 1), dtype=np.int64)
+    s = np.zeros(1, dtype=np.int64)
+    st = _load().orc_plan(_ptr(rows), _ptr(cols), _ptr(k), n, int(m), int(align), int(max_bucket),
+                          1 if literal else 0, off.ctypes.data, s.ctypes.data)
+    return st, off[:n].copy(), int(s[0])
+
+
+def place_fixed(rows, cols, k, m, align, s, literal=False):
+    """Greedy placement in planner order at one fixed slice size s.
+    Returns (placed?, offsets in input order)."""
+    rows, cols, k = _i64(rows), _i64(cols), _i64(k)
+    off = np.zeros(max(rows.size, 1), dtype=np.int64)
+    ok = _load().orc_place_fixed(_ptr(rows), _ptr(cols), _ptr(k), rows.size, int(m), int(align),
+                                 int(s), 1 if literal else 0, off.ctypes.data)
+    return bool(ok), off[:rows.size].copy()
+
+
+def planner_order(rows, cols, k):
+    """Input indices in planner order: block size descending, then element
+    count descending, then input position (plain numpy, for the tests)."""
+    rows, cols, k = _i64(rows), _i64(cols), _i64(k)
+    n, b = rows * cols, k * cols
+    return np.array(sorted(range(rows.size), key=lambda i: (-b[i], -n[i], i)), dtype=np.int64)
+
+
+def exists_placement(n_elems, b_elems, s, m, align):
+    """Exhaustive search: any placement of the tensors in this order at slice size s?"""
+    n, b = _i64(n_elems), _i64(b_elems)
+    return bool(_load().orc_exists_placement(_ptr(n), _ptr(b), n.size, int(s), int(m), int(align)))
+
+
+def bruteforce_min_bucket(rows, cols, k, m, align):
+    """True minimum bucket size over every order and placement (tiny inputs)."""
+    rows, cols, k = _i64(rows), _i64(cols), _i64(k)
+    return int(_load().orc_bruteforce_min_bucket(_ptr(rows), _ptr(cols), _ptr(k), rows.size,
+                                                 int(m), int(align)))
+
+
+def check_layout(rows, cols, k, m, align, offsets, s):
+    """Bit mask of broken layout rules (0 = valid); see oracle.cpp."""
+    rows, cols, k, off = _i64(rows), _i64(cols), _i64(k), _i64(offsets)
+    return int(_load().orc_check_layout(_ptr(rows), _ptr(cols), _ptr(k), rows.size, int(m),
+                                        int(align), _ptr(off), int(s)))
+
+
+def blocks(rows, cols, k, offsets):
+    """Quantisation blocks of a planned bucket, numbered in bucket order
+    (tensors by ascending offset, blocks in row order inside a tensor).
+
+    RaggedShard's unit (paper Sec. 3): k whole rows, the last block of a tensor
+    may be shorter.  Returns (start, length) int64 arrays.
+    """
+    rows, cols, k, off = _i64(rows), _i64(cols), _i64(k), _i64(offsets)
+    starts, lens = [], []
+    for i in np.argsort(off, kind="stable"):
+        n, b = int(rows[i] * cols[i]), int(k[i] * cols[i])
+        nb = -(-n // b)
+        st = int(off[i]) + b * np.arange(nb, dtype=np.int64)
+        ln = np.full(nb, b, dtype=np.int64)
+        ln[-1] = n - b * (nb - 1)
+        starts.append(st)
+        lens.append(ln)
+    if not starts:
+        return np.zeros(0, np.int64), np.zeros(0, np.int64)
+    return np.concatenate(starts), np.concatenate(lens)
+
+
+def padding_mask(rows, cols, offsets, bucket):
+    """Boolean mask of bucket elements that belong to no tensor."""
+    mask = np.ones(bucket, dtype=bool)
+    for r, c, o in zip(_i64(rows), _i64(cols), _i64(offsets)):
+        mask[int(o):int(o) + int(r * c)] = False
+    return mask
+
+
+# ---------------------------------------------------------------- update ---
+
+def step_scalars(lr, beta1, beta2, eps, wd, t):
+    """(b1, 1-b1, b2, 1-b2, sqrt(1-b2^t), eps, lr/(1-b1^t), 1-lr*wd) as float32."""
+    out = np.zeros(8, dtype=np.float32)
+    _load().orc_step_scalars(lr, beta1, beta2, eps, wd, int(t), out.ctypes.data)
+    return out
+
+
+def adam8_step(start, length, sidx, p, g_bits, mq, vq, scale_m, scale_v, pb_bits, hp, t,
+               grad_scale, threads=1):
+    """Block-wise 8-bit Adam (the 8-bit Adam case study, paper Sec. 6.3: each
+    device quantises its own blocks) over the listed blocks, in place.
+
+    p float32, g_bits uint16 (bf16), mq int8, vq uint8, pb_bits uint16 are
+    indexed by bucket element; scale_m/scale_v float32 by sidx[j].
+    """
+    start, length, sidx = _i64(start), _i64(length), _i64(sidx)
+    assert p.dtype == np.float32 and g_bits.dtype == np.uint16 and pb_bits.dtype == np.uint16
+    assert mq.dtype == np.int8 and vq.dtype == np.uint8
+    assert scale_m.dtype == np.float32 and scale_v.dtype == np.float32
+    for a in (p, g_bits, mq, vq, scale_m, scale_v, pb_bits):
+        assert a.flags.c_contiguous
+    if start.size:
+        hi = int(np.max(start + length))
+        assert hi <= min(p.size, g_bits.size, mq.size, vq.size, pb_bits.size)
+        assert int(np.max(sidx)) < min(scale_m.size, scale_v.size)
+    _load().orc_adam8_step(start.size, _ptr(start), _ptr(length), _ptr(sidx), _ptr(p), _ptr(g_bits),
+                           _ptr(mq), _ptr(vq), _ptr(scale_m), _ptr(scale_v), _ptr(pb_bits),
+                           hp["lr"], hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"], int(t),
+                           float(grad_scale), int(threads))
+
+
+def pack(src_bits, dst_bits, scale):
+    """Copy-in of the row-wise FSDP baseline: dst = bf16(float(src) * scale)."""
+    assert src_bits.dtype == np.uint16 and dst_bits.dtype == np.uint16
+    assert dst_bits.size >= src_bits.size and dst_bits.flags.c_contiguous
+    src = np.ascontiguousarray(src_bits)
+    _load().orc_pack(src.size, _ptr(src), _ptr(dst_bits), float(scale))
+
+
+def bf16_round(x):
+    """float32 -> bf16 bits, round to nearest even."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.size, dtype=np.uint16)
+    _load().orc_bf16_round(x.size, _ptr(x), _ptr(out))
+    return out
+
+
+class Bucket:
+    """Whole-bucket state on the host, stepped by the oracle.
+
+    Arrays follow the DBuffer picture (paper Sec. 5): one flat buffer per
+    kind, tensors are slices at their planned offsets.  Padding holds zeros;
+    the bf16 copy of padding is set to zero on every step.
+    """
+
+    def __init__(self, rows, cols, k, offsets, s, m):
+        self.rows, self.cols, self.k = _i64(rows), _i64(cols), _i64(k)
+        self.offsets = _i64(offsets)
+        self.s, self.m = int(s), int(m)
+        self.size = self.s * self.m
+        self.start, self.length = blocks(self.rows, self.cols, self.k, self.offsets)
+        self.sidx = np.arange(self.start.size, dtype=np.int64)
+        self.pad = padding_mask(self.rows, self.cols, self.offsets, self.size)
+        S, B = self.size, self.start.size
+        self.p = np.zeros(S, np.float32)
+        self.g = np.zeros(S, np.uint16)
+        self.mq = np.zeros(S, np.int8)
+        self.vq = np.zeros(S, np.uint8)
+        self.pb = np.zeros(S, np.uint16)
+        self.scale_m = np.zeros(B, np.float32)
+        self.scale_v = np.zeros(B, np.float32)
+
+    def tensor_slice(self, i):
+        o = int(self.offsets[i])
+        return slice(o, o + int(self.rows[i] * self.cols[i]))
+
+    def step(self, hp, t, grad_scale, threads=1):
+        adam8_step(self.start, self.length, self.sidx, self.p, self.g, self.mq, self.vq,
+                   self.scale_m, self.scale_v, self.pb, hp, t, grad_scale, threads)
+        self.pb[self.pad] = 0

@@ -1,0 +1,181 @@
+"""Tensor lists of the synthetic bucket workloads.
+
+Each tensor is (rows, cols, k): a row-major matrix cut into quantisation
+blocks of k whole rows (a 1-D tensor of length L is rows=L, cols=1, k=L, i.e.
+one block).  Shapes follow the workloads the veScale-FSDP pages evaluate on:
+a Llama-style dense layer, a GPT-OSS-style MoE layer, a ragged mix of block
+granularities, and a bucket whose gradients live in separate per-tensor
+allocations.  Nothing here is optimizer or planner arithmetic.
+"""
+import math
+from dataclasses import dataclass, field
+from typing import List
+
+import numpy as np
+
+from .rng import STREAM_SHAPES, stream_key, uniform_f64
+
+# Adam hyper-parameters of every workload (lr, beta1, beta2, eps, weight decay).
+HPARAMS = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01)
+PARAM_SIGMA = 0.02      # master weights ~ N(0, 0.02), fp32
+GRAD_SIGMA = 1e-3       # gradients ~ N(0, 1e-3), rounded to bf16
+
+
+@dataclass
+class TensorSpec:
+    name: str
+    rows: int
+    cols: int
+    k: int
+
+    @property
+    def numel(self):
+        return self.rows * self.cols
+
+
+@dataclass
+class Workload:
+    name: str
+    tensors: List[TensorSpec]
+    m: int                      # simulated ranks (equal slices of the bucket)
+    seed: int
+    steps: int = 10
+    align: int = 16
+    description: str = ""
+    extra: dict = field(default_factory=dict)
+
+    @property
+    def numel(self):
+        return sum(t.numel for t in self.tensors)
+
+    def arrays(self):
+        """(rows, cols, k) as three int64 numpy arrays in tensor order."""
+        r = np.array([t.rows for t in self.tensors], dtype=np.int64)
+        c = np.array([t.cols for t in self.tensors], dtype=np.int64)
+        k = np.array([t.k for t in self.tensors], dtype=np.int64)
+        return r, c, k
+
+
+def _vec(name, n):
+    return TensorSpec(name, n, 1, n)
+
+
+def tiny(m=4):
+    """W[512,256] in 16-row blocks, bias[512] and LayerNorm w[256] as single blocks."""
+    return Workload("tiny_m4", [TensorSpec("W", 512, 256, 16), _vec("bias", 512), _vec("ln_w", 256)],
+                    m=m, seed=0, steps=10,
+                    description="W[512,256] k=16, bias[512], LN[256]; m=4; 10 steps")
+
+
+LLAMA_SHAPES = [("wq", 4096, 4096), ("wk", 1024, 4096), ("wv", 1024, 4096), ("wo", 4096, 4096),
+                ("gate", 14336, 4096), ("up", 14336, 4096), ("down", 14336, 4096)]
+
+
+def _llama_tensors(prefix=""):
+    ts = [TensorSpec(prefix + n, r, c, 1) for n, r, c in LLAMA_SHAPES]
+    # RMSNorm weights: one row of 4096, block = that row.
+    ts += [TensorSpec(prefix + "norm1", 1, 4096, 1), TensorSpec(prefix + "norm2", 1, 4096, 1)]
+    return ts
+
+
+def llama_layer(m=8):
+    return Workload("llama_layer_m8", _llama_tensors(), m=m, seed=1, steps=10,
+                    description="Llama layer h=4096, GQA 32q/8kv, SwiGLU 14336; 1-row blocks; m=8")
+
+
+def moe_layer(m=64):
+    ts = []
+    for e in range(32):
+        ts.append(TensorSpec(f"e{e}.gate_up", 5760, 2880, 16))
+        ts.append(TensorSpec(f"e{e}.down", 2880, 2880, 16))
+    ts.append(TensorSpec("router", 32, 2880, 1))
+    ts += [TensorSpec("attn_q", 4096, 2880, 1), TensorSpec("attn_o", 4096, 2880, 1),
+           TensorSpec("attn_k", 512, 2880, 1), TensorSpec("attn_v", 512, 2880, 1)]
+    return Workload(f"moe_layer_m{m}", ts, m=m, seed=2, steps=10,
+                    description="MoE layer h=2880, 32 experts (gate_up 5760x2880, down 2880x2880, "
+                                "16-row blocks), router, attention (1-row blocks)")
+
+
+STRESS_COLS = (1, 1024, 2880, 4096, 7168)
+STRESS_KS = (1, 8, 16, 128)
+
+
+def ragged_stress(m=8, n_tensors=400, target=1_000_000_000, seed=3):
+    """400 tensors, rows log-uniform in [64, 16384], cols and k uniform from
+    fixed sets, rows rescaled so the bucket holds ~1.0e9 parameters.
+
+    The literal draw averages ~3.5e9 parameters, so rows are multiplied by a
+    common factor (iterated until the total is within 0.01% of the target),
+    rounded and clamped back to [64, 16384].  k is capped at rows.
+    """
+    u = uniform_f64(stream_key(seed, STREAM_SHAPES), 0, 3 * n_tensors).reshape(n_tensors, 3)
+    lo, hi = math.log(64.0), math.log(16384.0)
+    rows0 = np.exp(lo + u[:, 0] * (hi - lo))
+    cols = np.array([STRESS_COLS[min(int(x * 5), 4)] for x in u[:, 1]], dtype=np.int64)
+    ks = np.array([STRESS_KS[min(int(x * 4), 3)] for x in u[:, 2]], dtype=np.int64)
+    f = target / float(np.sum(rows0 * cols))
+    rows = None
+    for _ in range(50):
+        rows = np.clip(np.rint(rows0 * f), 64, 16384).astype(np.int64)
+        tot = int(np.sum(rows * cols))
+        if abs(tot - target) <= 1e-4 * target:
+            break
+        f *= target / tot
+    ts = [TensorSpec(f"t{i}", int(rows[i]), int(cols[i]), int(min(ks[i], rows[i])))
+          for i in range(n_tensors)]
+    return Workload(f"ragged_stress_m{m}", ts, m=m, seed=seed, steps=10,
+                    description="400 tensors, rows log-uniform [64,16384], cols in "
+                                "{1,1024,2880,4096,7168}, k in {1,8,16,128}; ~1.0e9 params")
+
+
+def copyin(n_tensors=200, m=64):
+    """Llama-layer shapes cycled (wq, wk, wv, wo, gate, up, down, norm1, norm2, ...)."""
+    base = _llama_tensors()
+    ts = []
+    for i in range(n_tensors):
+        b = base[i % len(base)]
+        ts.append(TensorSpec(f"L{i // len(base)}.{b.name}", b.rows, b.cols, b.k))
+    return Workload(f"copyin_{n_tensors}_m{m}", ts, m=m, seed=4, steps=20,
+                    description=f"Llama-layer shapes cycled to {n_tensors} tensors; grads in "
+                                f"{n_tensors} separate allocations; m={m}")
+
+
+def ragged_mix(m=4, seed=5):
+    """Moderate bucket that crosses every code path: per-element blocks,
+    8-element blocks, single odd blocks, row blocks below and far above one
+    tile, partial last blocks, odd lengths."""
+    ts = [
+        TensorSpec("vec_b1", 1000, 1, 1),
+        TensorSpec("vec_b8", 777, 1, 8),
+        _vec("vec_odd", 333),
+        TensorSpec("rows48", 300, 48, 16),
+        TensorSpec("exp_gu", 129, 2880, 16),
+        TensorSpec("big128", 260, 1024, 128),
+        TensorSpec("row7168", 5, 7168, 1),
+        TensorSpec("odd4099", 1, 4099, 1),
+        TensorSpec("b300", 13, 100, 3),
+        TensorSpec("small", 2, 3, 1),
+        _vec("vec4097", 4097),
+        TensorSpec("huge_blk", 40, 7168, 40),
+    ]
+    return Workload(f"ragged_mix_m{m}", ts, m=m, seed=seed, steps=4,
+                    description="ragged mix of block granularities 1..286720 elements")
+
+
+_BUILDERS = {
+    "tiny_m4": lambda: tiny(4),
+    "llama_layer_m8": lambda: llama_layer(8),
+    "moe_layer_m64": lambda: moe_layer(64),
+    "ragged_stress_m8": lambda: ragged_stress(8),
+    "ragged_stress_m128": lambda: ragged_stress(128),
+    "ragged_stress_m1024": lambda: ragged_stress(1024),
+    "copyin_200_m64": lambda: copyin(200, 64),
+    "copyin_9_m64": lambda: copyin(9, 64),
+    "ragged_mix_m4": lambda: ragged_mix(4),
+    "ragged_mix_m8": lambda: ragged_mix(8),
+}
+WORKLOAD_NAMES = tuple(_BUILDERS)
+
+
+def workload(name):
+    return _BUILDERS[name]()

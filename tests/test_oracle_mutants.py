@@ -1,0 +1,83 @@
+"""Plant plausible mistakes in a copy of the oracle and check that its pins
+fail (CPU only).
+
+Each case rewrites one line of a temporary copy of ``oracle/oracle.cpp``
+(a flipped sign, a dropped term, a swapped operand, a wrong rounding or
+layout rule), rebuilds it there, and runs the pin test that must catch it.
+The real oracle is never modified.
+"""
+import os
+import shutil
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+# name: (original line(s), planted mistake, pin test that must fail)
+MUTANTS = {
+    "m_sign": ("        m = m + t;", "        m = m - t;",
+               "test_oracle_adam.py::test_golden_first_step"),
+    "no_decay": ("        float pn = p[i] * c.decay;", "        float pn = p[i];",
+                 "test_oracle_adam.py::test_golden_first_step"),
+    "no_bias_corr2": ("        float d = r / c.bc2s;", "        float d = r;",
+                      "test_oracle_adam.py::test_golden_first_step"),
+    "eps_inside_sqrt": ("        float r = std::sqrt(v);\n        float d = r / c.bc2s;\n        d = d + c.eps;",
+                        "        float r = std::sqrt(v);\n        float d = std::sqrt(v + c.eps) / c.bc2s;",
+                        "test_oracle_adam.py::test_first_step_closed_form"),
+    "m_dequant_255": ("    const float dqm = *sm / 127.0f;", "    const float dqm = *sm / 255.0f;",
+                      "test_oracle_adam.py::test_uniform_magnitude_blocks_reduce_to_adamw"),
+    "v_quant_127": ("    const float qv = amax_r > 0.0f ? 255.0f / amax_r : 0.0f;",
+                    "    const float qv = amax_r > 0.0f ? 127.0f / amax_r : 0.0f;",
+                    "test_oracle_adam.py::test_golden_first_step"),
+    "truncate_codes": ("        float a = std::rint(mt[i] * qm);", "        float a = std::trunc(mt[i] * qm);",
+                       "test_oracle_adam.py::test_first_step_codes_are_nearest_levels"),
+    "v_not_squared": ("        float vo = so * so;", "        float vo = so;",
+                      "test_oracle_adam.py::test_uniform_magnitude_blocks_reduce_to_adamw"),
+    "beta_swap": ("        float m = c.b1 * mo;", "        float m = c.b2 * mo;",
+                  "test_oracle_adam.py::test_uniform_magnitude_blocks_reduce_to_adamw"),
+    "no_bias_corr1": ("    c.step = (float)(l / bc1);", "    c.step = (float)(l);",
+                      "test_oracle_adam.py::test_first_step_closed_form"),
+    "coupled_decay": ("        float gi = bf16_to_f32(g[i]) * grad_scale;",
+                      "        float gi = bf16_to_f32(g[i]) * grad_scale + 0.01f * p[i];",
+                      "test_oracle_adam.py::test_first_step_closed_form"),
+    "scale_not_absmax": ("    *sm = amax_m;", "    *sm = amax_m * 0.5f;",
+                         "test_oracle_adam.py::test_first_step_codes_are_nearest_levels"),
+    "bf16_truncates": ("    u += 0x7FFFu + ((u >> 16) & 1u);", "    u += 0;",
+                       "test_oracle_adam.py::test_bf16_rounding_matches_torch"),
+    "walk_skips_check": ("        if (j > 0 && start_allowed(R - j, n, b, s, m, A)) return R - j;",
+                         "        if (j > 0) return R - j;",
+                         "test_oracle_layout.py::test_greedy_places_iff_any_placement_exists"),
+    "skip_rule_too_strong": ("        if (t.n > 2 * s && s % t.b != 0) return false;",
+                             "        if (t.n > s && s % t.b != 0) return false;",
+                             "test_oracle_layout.py::test_chosen_slice_is_smallest_feasible"),
+    "sort_ascending": ("        if (x.b != y.b) return x.b > y.b;", "        if (x.b != y.b) return x.b < y.b;",
+                       "test_oracle_layout.py::test_golden_tiny_layout"),
+    "candidate_step_b": ("    const int64_t L = std::lcm(A, b);", "    const int64_t L = b;",
+                         "test_oracle_layout.py::test_literal_scan_equals_walk"),
+    "edge_counts_as_inside": ("    for (int64_t r = o / s + 1; r < m && r * s < o + n; ++r)",
+                              "    for (int64_t r = o / s + 1; r < m && r * s <= o + n; ++r)",
+                              "test_oracle_layout.py::test_literal_scan_equals_walk"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pin_catches_planted_mistake(name, tmp_path):
+    orig, bad, pin = MUTANTS[name]
+    src = open(os.path.join(ROOT, "oracle", "oracle.cpp")).read()
+    assert src.count(orig) == 1, f"mutation site of {name} not found once"
+    work = tmp_path / "repo"
+    os.makedirs(work / "tests")
+    shutil.copytree(os.path.join(ROOT, "oracle"), work / "oracle",
+                    ignore=shutil.ignore_patterns("*.so", "__pycache__"))
+    shutil.copytree(os.path.join(ROOT, "synth"), work / "synth",
+                    ignore=shutil.ignore_patterns("__pycache__"))
+    for f in ("conftest.py", "test_oracle_adam.py", "test_oracle_layout.py"):
+        shutil.copy(os.path.join(ROOT, "tests", f), work / "tests" / f)
+    shutil.copytree(os.path.join(ROOT, "tests", "golden"), work / "tests" / "golden")
+    (work / "oracle" / "oracle.cpp").write_text(src.replace(orig, bad))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+                        "tests/" + pin], cwd=work, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 1 and "failed" in r.stdout, (
+        f"pin {pin} did not catch mutant {name}:\n{r.stdout[-2000:]}{r.stderr[-2000:]}")
