@@ -1,0 +1,200 @@
+/*
+ * dbuf.h -- C-ABI of the ragged-bucket optimizer step for B200 (sm_100a).
+ *
+ * What the library does (veScale-FSDP: Flexible and High-Performance FSDP at
+ * Scale, MLSys 2026, as the notes.yuuk.io and gist.science pages summarise
+ * it):
+ *
+ *   RaggedShard (paper Sec. 3, page section "1. RaggedShard"): every tensor is
+ *     cut into whole blocks of k rows; a block is the unit of block-wise
+ *     quantisation and never straddles two devices' shards.
+ *   Structure-aware planning (paper Sec. 4, page section "2. Structure-aware
+ *     planning algorithm"): the tensors of one communication bucket are sorted
+ *     by block size, largest first, and given offsets so that every boundary
+ *     between the m equal per-device slices falls on a block edge, with
+ *     padding only between tensors.  Runs once, on the host.
+ *   DBuffer (paper Sec. 5, page section "3. DBuffer"): the bucket is one flat
+ *     buffer per kind (batch-allocated once); tensors are zero-copy views;
+ *     group-level operations run once over the whole bucket instead of once
+ *     per tensor; streams are ordered explicitly (no record_stream).
+ *   8-bit Adam case study (paper Sec. 6.3): block-wise quantised optimizer
+ *     states, each device quantising its own blocks with no communication.
+ *
+ * Conventions of every entry point:
+ *   - Status codes are returned; on failure dbuf_last_error() gives a
+ *     thread-local message.  Nothing aborts the process.
+ *   - "stream" is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Device work is enqueued on it and is asynchronous; no entry
+ *     point synchronises except dbuf_get_device_status and
+ *     dbuf_adam8_step_host's callers' own sync.  record_stream is never used.
+ *   - Device calls must be made with the device that created the dbuf
+ *     current; otherwise DBUF_EINVAL.
+ *   - A dbuf is not safe for concurrent calls from several host threads.
+ *   - Element offsets are in elements of the array in question; the bucket
+ *     holds m*s elements of each kind, s = slice size.
+ */
+#ifndef DBUF_H
+#define DBUF_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A tensor of the bucket: row-major rows x cols, quantisation block = k whole
+ * rows (the last block may be shorter).  A 1-D tensor of length L is
+ * rows=L, cols=1, k=L (one block).  Requires rows, cols, k >= 1, k <= rows. */
+typedef struct {
+    int64_t rows, cols, k;
+} dbuf_tensor_desc;
+
+typedef struct dbuf_plan_s dbuf_plan_t; /* host-only layout, owned by the caller */
+typedef struct dbuf_s dbuf_t;           /* device bucket, owned by the caller   */
+
+typedef enum {
+    DBUF_OK = 0,
+    DBUF_EINVAL = 1,      /* bad argument (message says which)                 */
+    DBUF_EINFEASIBLE = 2, /* no layout within max_bucket_elems                 */
+    DBUF_ENOMEM = 3,      /* host or device allocation failed                  */
+    DBUF_ECUDA = 4,       /* a CUDA runtime call failed (message has the name) */
+    DBUF_EDEVICE = 5      /* a kernel reported an error in its status word     */
+} dbuf_status;
+
+/* Plan the layout of one bucket (host only, no CUDA).
+ *   descs[n]          tensors in the caller's order (copied; not retained)
+ *   m                 number of equal slices (devices), >= 1
+ *   align_elems       every tensor start and s are multiples of it, >= 1;
+ *                     dbuf_create needs a multiple of 16 (128-bit accesses)
+ *   max_bucket_elems  0 = no cap; otherwise m*s above it -> DBUF_EINFEASIBLE
+ * Order: block size k*cols descending, then element count descending, then
+ * input position.  s is the smallest multiple of align_elems, at least
+ * ceil(sum/m), for which earliest-start placement in that order puts every
+ * tensor so that each slice boundary inside a tensor is on a block edge.
+ * n = 0 gives an empty plan (s = 0).  *out is NULL on failure. */
+dbuf_status dbuf_plan(const dbuf_tensor_desc* descs, int32_t n, int32_t m, int64_t align_elems,
+                      int64_t max_bucket_elems, dbuf_plan_t** out);
+
+/* Read a plan.  Any output pointer may be NULL.  offsets[n] (caller-owned)
+ * receives each tensor's start in the caller's order.  n_blocks counts the
+ * quantisation blocks; blocks are numbered in bucket order (tensors by
+ * ascending offset, blocks in row order), which is the index of their
+ * scales. */
+dbuf_status dbuf_plan_info(const dbuf_plan_t* plan, int64_t* slice_elems, int64_t* bucket_elems,
+                           int64_t* padding_elems, int64_t* n_blocks, int64_t* offsets);
+
+void dbuf_plan_free(dbuf_plan_t* plan); /* NULL is a no-op */
+
+/* Bytes of device memory dbuf_create needs for this plan (one allocation:
+ * fp32 master, bf16 param, bf16 grad, int8 m codes, uint8 sqrt(v) codes,
+ * per-block scales, work tables, status word), 256-byte aligned parts.
+ * 0 if plan is NULL. */
+size_t dbuf_required_bytes(const dbuf_plan_t* plan);
+
+/* Create the device bucket of a plan (the plan is copied; it may be freed
+ * afterwards).  device_base = NULL: one cudaMalloc of dbuf_required_bytes,
+ * freed by dbuf_destroy.  Otherwise the caller's device memory, at least
+ * dbuf_required_bytes long (base_bytes says how long) and 256-byte aligned;
+ * it stays the caller's.  The whole region is zeroed on `stream` and the
+ * work tables are copied in, both asynchronously: the bucket is ready for
+ * work ordered after them on that stream.  DBUF_EINVAL if the plan's
+ * alignment is not a multiple of 16. */
+dbuf_status dbuf_create(const dbuf_plan_t* plan, void* device_base, size_t base_bytes, void* stream,
+                        dbuf_t** out);
+
+/* Copy-in gather, the per-parameter copy of row-wise FSDP that the
+ * zero-copy bucket removes (page section "Importance of zero-copy
+ * communication"): for every tensor i,
+ *   grad[offset_i + j] = bf16(float(grads_bf16[i][j]) * scale), j < rows*cols.
+ * grads_bf16[n] are device pointers in the caller's order (host array,
+ * read during the call only); the device memory they point to must stay
+ * valid until the copy completes on `stream`.  Padding is not touched. */
+dbuf_status dbuf_pack_grads(dbuf_t* db, const void* const* grads_bf16, float scale, void* stream);
+
+typedef struct {
+    float lr, beta1, beta2, eps, weight_decay;
+    int64_t step; /* 1-based step number t used in the bias corrections */
+} dbuf_adam_hparams;
+
+/* One block-wise 8-bit Adam step over the whole bucket, zero-copy: reads the
+ * bf16 gradient bucket in place, one grouped kernel launch.  Per element
+ * (fp32, each operation rounded separately, in this order):
+ *   g = grad * grad_scale;  m_old = qm * scale_m / 127;  s = qv * scale_v / 255;
+ *   m = b1*m_old + (1-b1)*g;  v = b2*s*s + (1-b2)*g*g;  r = sqrt(v);
+ *   p = p*(1 - lr*wd) - (lr/(1-b1^t)) * m / (r/sqrt(1-b2^t) + eps);
+ *   param_bf16 = round-to-nearest-even(p)
+ * per block: scale_m = max|m|, scale_v = max r, qm = rint(m*127/scale_m)
+ * clamped to [-127,127], qv = rint(r*255/scale_v) clamped to [0,255] (codes
+ * 0 where the scale is 0).  Per-step scalars are formed in double, rounded to
+ * float once.  The bf16 param bucket is set to 0 on every padding element.
+ * grad_scale is typically 1/m (the reduce-scatter average). */
+dbuf_status dbuf_adam8_step(dbuf_t* db, const dbuf_adam_hparams* hp, float grad_scale, void* stream);
+
+/* The same step with host buffers at both ends (the end-to-end path): copies
+ * grads_host (bucket_elems bf16, caller's host memory, pinned for overlap)
+ * into the grad bucket, runs dbuf_adam8_step, and copies the bf16 param
+ * bucket back to params_bf16_host (bucket_elems bf16).  All three are
+ * enqueued on `stream`; the caller synchronises before reading the output. */
+dbuf_status dbuf_adam8_step_host(dbuf_t* db, const dbuf_adam_hparams* hp, float grad_scale,
+                                 const void* grads_host, void* params_bf16_host, void* stream);
+
+typedef enum {
+    DBUF_MASTER_F32 = 0, /* float  */
+    DBUF_PARAM_BF16 = 1, /* bf16   (the all-gather buffer) */
+    DBUF_GRAD_BF16 = 2,  /* bf16   (the reduce-scatter buffer) */
+    DBUF_M_I8 = 3,       /* int8   codes of m */
+    DBUF_V_U8 = 4        /* uint8  codes of sqrt(v) */
+} dbuf_which;
+
+typedef struct {
+    void* ptr; /* device pointer to the tensor's first element */
+    int64_t rows, cols, offset_elems;
+} dbuf_view;
+
+/* Zero-copy views: out[n] (caller-owned) gets each tensor's place in the
+ * chosen bucket array, in the caller's tensor order.  Pure pointer
+ * arithmetic; pointers are borrowed and valid until dbuf_destroy. */
+dbuf_status dbuf_unpack_views(const dbuf_t* db, dbuf_which which, dbuf_view* out);
+
+/* Whole bucket array of one kind (e.g. for an in-place all-gather or
+ * reduce-scatter of slice r = [r*s, (r+1)*s)).  Borrowed pointer. */
+dbuf_status dbuf_bucket(const dbuf_t* db, dbuf_which which, void** ptr, int64_t* elems);
+
+/* Per-block scales, interleaved: scales[2j] = scale of m, scales[2j+1] =
+ * scale of sqrt(v), for block j in bucket order.  Borrowed device pointer. */
+dbuf_status dbuf_scales(const dbuf_t* db, float** scales, int64_t* n_blocks);
+
+/* Read (and synchronise `stream` for) the device status word that the
+ * kernels set instead of trapping: 0 = fine; 1 = a bounded wait on a copy
+ * ran out; 2 = a work-table entry was out of range; 3 = a copy-in source
+ * pointer was not 2-byte aligned. */
+dbuf_status dbuf_get_device_status(dbuf_t* db, int32_t* code, void* stream);
+
+/* One entry of the step kernel's work table (introspection for tests and
+ * tools; the kernel's own table holds the same entries).  kind 0: up to 256
+ * whole blocks of one tensor, at most 4096 elements counted from the
+ * 16-element boundary at or below first_elem; kind 1: one block longer than
+ * that, streamed twice; kind 2: a padding range whose bf16 copy is zeroed. */
+typedef struct {
+    int64_t first_elem, first_block, n_elems;
+    int32_t block_elems, kind, n_blocks, reserved;
+} dbuf_work_item;
+
+/* Copy the work table that dbuf_create would build for `plan` into out[cap]
+ * (host memory; may be NULL when cap = 0) and its length into *n. */
+dbuf_status dbuf_work_table(const dbuf_plan_t* plan, dbuf_work_item* out, int64_t cap, int64_t* n);
+
+/* Set the status word back to 0 (asynchronous, on `stream`). */
+dbuf_status dbuf_clear_device_status(dbuf_t* db, void* stream);
+
+void dbuf_destroy(dbuf_t* db); /* NULL is a no-op; frees only what it allocated */
+
+/* Message of the last failure on this host thread ("" if none). */
+const char* dbuf_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DBUF_H */

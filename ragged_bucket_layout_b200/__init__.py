@@ -1,0 +1,283 @@
+"""Python binding of libdbuf, the B200 ragged-bucket 8-bit Adam library.
+
+Argument marshalling only: every step of the path (planning, the bucket step,
+the copy-in, the padding zeroing) runs in the C++/CUDA library, whose C-ABI is
+declared in ``include/dbuf.h``; this module gives the same entry points the
+same names.  ``DBuffer`` adds PyTorch views of a bucket whose device memory
+PyTorch allocated (PyTorch is used for memory and streams only).
+
+There is no fallback: importing this package without a built ``libdbuf.so``
+raises ImportError.
+"""
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdbuf.so")
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is not built; run `python -c 'import __graft_entry__ as g; g.build()'` "
+        "or `python ragged_bucket_layout_b200/build.py`")
+_lib = ctypes.CDLL(LIB_PATH)
+
+DBUF_OK, DBUF_EINVAL, DBUF_EINFEASIBLE, DBUF_ENOMEM, DBUF_ECUDA, DBUF_EDEVICE = range(6)
+DBUF_MASTER_F32, DBUF_PARAM_BF16, DBUF_GRAD_BF16, DBUF_M_I8, DBUF_V_U8 = range(5)
+_STATUS_NAMES = {0: "DBUF_OK", 1: "DBUF_EINVAL", 2: "DBUF_EINFEASIBLE", 3: "DBUF_ENOMEM",
+                 4: "DBUF_ECUDA", 5: "DBUF_EDEVICE"}
+
+
+class DbufError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__(f"{_STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+class dbuf_tensor_desc(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int64), ("cols", ctypes.c_int64), ("k", ctypes.c_int64)]
+
+
+class dbuf_adam_hparams(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
+                ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float), ("step", ctypes.c_int64)]
+
+
+class dbuf_view(ctypes.Structure):
+    _fields_ = [("ptr", ctypes.c_void_p), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("offset_elems", ctypes.c_int64)]
+
+
+class dbuf_work_item(ctypes.Structure):
+    _fields_ = [("first_elem", ctypes.c_int64), ("first_block", ctypes.c_int64), ("n_elems", ctypes.c_int64),
+                ("block_elems", ctypes.c_int32), ("kind", ctypes.c_int32), ("n_blocks", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
+_P, _PP = ctypes.c_void_p, ctypes.POINTER(ctypes.c_void_p)
+_i32, _i64, _f32, _sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+_pi64 = ctypes.POINTER(ctypes.c_int64)
+_SIGS = {
+    "dbuf_plan": (ctypes.c_int, [ctypes.POINTER(dbuf_tensor_desc), _i32, _i32, _i64, _i64, _PP]),
+    "dbuf_plan_info": (ctypes.c_int, [_P, _pi64, _pi64, _pi64, _pi64, _pi64]),
+    "dbuf_plan_free": (None, [_P]),
+    "dbuf_required_bytes": (_sz, [_P]),
+    "dbuf_create": (ctypes.c_int, [_P, _P, _sz, _P, _PP]),
+    "dbuf_pack_grads": (ctypes.c_int, [_P, _PP, _f32, _P]),
+    "dbuf_adam8_step": (ctypes.c_int, [_P, ctypes.POINTER(dbuf_adam_hparams), _f32, _P]),
+    "dbuf_adam8_step_host": (ctypes.c_int, [_P, ctypes.POINTER(dbuf_adam_hparams), _f32, _P, _P, _P]),
+    "dbuf_unpack_views": (ctypes.c_int, [_P, ctypes.c_int, ctypes.POINTER(dbuf_view)]),
+    "dbuf_bucket": (ctypes.c_int, [_P, ctypes.c_int, _PP, _pi64]),
+    "dbuf_scales": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.POINTER(ctypes.c_float)), _pi64]),
+    "dbuf_get_device_status": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int32), _P]),
+    "dbuf_clear_device_status": (ctypes.c_int, [_P, _P]),
+    "dbuf_work_table": (ctypes.c_int, [_P, ctypes.POINTER(dbuf_work_item), _i64, _pi64]),
+    "dbuf_destroy": (None, [_P]),
+    "dbuf_last_error": (ctypes.c_char_p, []),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+EXPORTED = tuple(_SIGS)
+
+
+def dbuf_last_error():
+    return _lib.dbuf_last_error().decode()
+
+
+def _check(st):
+    if st != DBUF_OK:
+        raise DbufError(st, dbuf_last_error())
+
+
+def _stream(s):
+    if s is None:
+        return None
+    if hasattr(s, "cuda_stream"):
+        return ctypes.c_void_p(s.cuda_stream)
+    return ctypes.c_void_p(int(s))
+
+
+# ------------------------------------------------------------------ plans
+
+class Plan:
+    """Owner of a dbuf_plan_t (freed with dbuf_plan_free)."""
+
+    def __init__(self, handle, n):
+        self.handle = handle
+        self.n = n
+
+    def __del__(self):
+        if getattr(self, "handle", None):
+            _lib.dbuf_plan_free(self.handle)
+            self.handle = None
+
+
+def dbuf_plan(rows, cols, k, m, align_elems=16, max_bucket_elems=0):
+    n = len(rows)
+    descs = (dbuf_tensor_desc * max(n, 1))(*[dbuf_tensor_desc(int(r), int(c), int(q))
+                                             for r, c, q in zip(rows, cols, k)])
+    out = ctypes.c_void_p()
+    _check(_lib.dbuf_plan(descs, n, int(m), int(align_elems), int(max_bucket_elems), ctypes.byref(out)))
+    return Plan(out.value, n)
+
+
+def dbuf_plan_info(plan):
+    s, b, p, nb = (ctypes.c_int64() for _ in range(4))
+    offs = (ctypes.c_int64 * max(plan.n, 1))()
+    _check(_lib.dbuf_plan_info(plan.handle, ctypes.byref(s), ctypes.byref(b), ctypes.byref(p),
+                               ctypes.byref(nb), offs))
+    return dict(slice=s.value, bucket=b.value, padding=p.value, n_blocks=nb.value,
+                offsets=[offs[i] for i in range(plan.n)])
+
+
+def dbuf_plan_free(plan):
+    if plan.handle:
+        _lib.dbuf_plan_free(plan.handle)
+        plan.handle = None
+
+
+def dbuf_required_bytes(plan):
+    return int(_lib.dbuf_required_bytes(plan.handle))
+
+
+# ---------------------------------------------------------------- buckets
+
+def dbuf_create(plan, device_base=None, base_bytes=0, stream=None):
+    out = ctypes.c_void_p()
+    _check(_lib.dbuf_create(plan.handle, device_base, int(base_bytes), _stream(stream), ctypes.byref(out)))
+    return out.value
+
+
+def dbuf_destroy(db):
+    _lib.dbuf_destroy(db)
+
+
+def _hp(hp):
+    return dbuf_adam_hparams(hp["lr"], hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"], int(hp["step"]))
+
+
+def dbuf_pack_grads(db, grad_ptrs, scale, stream=None):
+    arr = (ctypes.c_void_p * max(len(grad_ptrs), 1))(*[int(p) for p in grad_ptrs])
+    _check(_lib.dbuf_pack_grads(db, arr, float(scale), _stream(stream)))
+
+
+def dbuf_adam8_step(db, hp, grad_scale, stream=None):
+    h = _hp(hp)
+    _check(_lib.dbuf_adam8_step(db, ctypes.byref(h), float(grad_scale), _stream(stream)))
+
+
+def dbuf_adam8_step_host(db, hp, grad_scale, grads_host_ptr, params_host_ptr, stream=None):
+    h = _hp(hp)
+    _check(_lib.dbuf_adam8_step_host(db, ctypes.byref(h), float(grad_scale), grads_host_ptr,
+                                     params_host_ptr, _stream(stream)))
+
+
+def dbuf_unpack_views(db, which, n):
+    out = (dbuf_view * max(n, 1))()
+    _check(_lib.dbuf_unpack_views(db, int(which), out))
+    return [(out[i].ptr or 0, out[i].rows, out[i].cols, out[i].offset_elems) for i in range(n)]
+
+
+def dbuf_bucket(db, which):
+    p, n = ctypes.c_void_p(), ctypes.c_int64()
+    _check(_lib.dbuf_bucket(db, int(which), ctypes.byref(p), ctypes.byref(n)))
+    return p.value or 0, n.value
+
+
+def dbuf_scales(db):
+    p, n = ctypes.POINTER(ctypes.c_float)(), ctypes.c_int64()
+    _check(_lib.dbuf_scales(db, ctypes.byref(p), ctypes.byref(n)))
+    return ctypes.cast(p, ctypes.c_void_p).value or 0, n.value
+
+
+def dbuf_get_device_status(db, stream=None):
+    code = ctypes.c_int32()
+    _check(_lib.dbuf_get_device_status(db, ctypes.byref(code), _stream(stream)))
+    return code.value
+
+
+def dbuf_work_table(plan):
+    """Work table of the step kernel as a list of dicts (host introspection)."""
+    n = ctypes.c_int64()
+    _check(_lib.dbuf_work_table(plan.handle, None, 0, ctypes.byref(n)))
+    arr = (dbuf_work_item * max(n.value, 1))()
+    _check(_lib.dbuf_work_table(plan.handle, arr, n.value, ctypes.byref(n)))
+    return [dict(first_elem=a.first_elem, first_block=a.first_block, n_elems=a.n_elems,
+                 block_elems=a.block_elems, kind=a.kind, n_blocks=a.n_blocks) for a in arr[:n.value]]
+
+
+def dbuf_clear_device_status(db, stream=None):
+    _check(_lib.dbuf_clear_device_status(db, _stream(stream)))
+
+
+# ----------------------------------------------------- PyTorch-owned buckets
+
+_DTYPES = None
+
+
+def _dtypes():
+    global _DTYPES
+    if _DTYPES is None:
+        import torch
+        _DTYPES = {DBUF_MASTER_F32: (torch.float32, 4), DBUF_PARAM_BF16: (torch.bfloat16, 2),
+                   DBUF_GRAD_BF16: (torch.bfloat16, 2), DBUF_M_I8: (torch.int8, 1), DBUF_V_U8: (torch.uint8, 1)}
+    return _DTYPES
+
+
+class DBuffer:
+    """A bucket whose single device allocation is a PyTorch uint8 tensor.
+
+    Views are slices of that tensor (zero-copy); all work goes through the
+    C-ABI calls above on the given (or current) CUDA stream.
+    """
+
+    def __init__(self, plan, device="cuda", stream=None):
+        import torch
+        self.plan = plan
+        self.info = dbuf_plan_info(plan)
+        nbytes = dbuf_required_bytes(plan)
+        self.base = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+        self.stream = stream if stream is not None else torch.cuda.current_stream(self.base.device)
+        self.handle = dbuf_create(plan, self.base.data_ptr(), self.base.numel(), self.stream)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            dbuf_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        self.close()
+
+    def _view(self, ptr, elems, which):
+        dt, es = _dtypes()[which]
+        off = ptr - self.base.data_ptr()
+        return self.base[off:off + elems * es].view(dt)
+
+    def array(self, which):
+        ptr, elems = dbuf_bucket(self.handle, which)
+        return self._view(ptr, elems, which)
+
+    def views(self, which):
+        out = []
+        for ptr, rows, cols, _ in dbuf_unpack_views(self.handle, which, self.plan.n):
+            out.append(self._view(ptr, rows * cols, which).view(rows, cols))
+        return out
+
+    def scales(self):
+        import torch
+        ptr, nb = dbuf_scales(self.handle)
+        off = ptr - self.base.data_ptr()
+        return self.base[off:off + nb * 8].view(torch.float32).view(nb, 2)
+
+    def step(self, hp, grad_scale):
+        dbuf_adam8_step(self.handle, hp, grad_scale, self.stream)
+
+    def step_host(self, hp, grad_scale, grads_host_ptr, params_host_ptr):
+        dbuf_adam8_step_host(self.handle, hp, grad_scale, grads_host_ptr, params_host_ptr, self.stream)
+
+    def pack(self, grads, scale):
+        dbuf_pack_grads(self.handle, [g.data_ptr() for g in grads], scale, self.stream)
+
+    def device_status(self):
+        return dbuf_get_device_status(self.handle, self.stream)

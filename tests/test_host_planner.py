@@ -1,0 +1,194 @@
+"""Host-side logic of the product library (CPU only, no device calls).
+
+* libdbuf.so loads and exports every entry point include/dbuf.h declares;
+* the C++ planner (dbuf_plan) gives the oracle's layout bit for bit: on every
+  workload bucket and on thousands of random small buckets;
+* invalid descriptors and caps come back as status codes, not crashes;
+* dbuf_required_bytes covers every bucket array.
+"""
+import os
+import random
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+import ragged_bucket_layout_b200 as rb
+import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_entry_points():
+    hdr = open(os.path.join(ROOT, "include", "dbuf.h")).read()
+    hdr = re.sub(r"/\*.*?\*/", "", hdr, flags=re.S)
+    return sorted(set(re.findall(r"\b(dbuf_[a-z0-9_]+)\s*\(", hdr)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_entry_points()
+    assert len(names) >= 15
+    out = subprocess.run(["nm", "-D", "--defined-only", rb.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\bT (\w+)", out))
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    assert set(rb.EXPORTED) == set(names)
+
+
+def test_oracle_and_library_share_nothing():
+    """The oracle library exports none of the product's symbols and the
+    product none of the oracle's."""
+    prod = subprocess.run(["nm", "-D", "--defined-only", rb.LIB_PATH], capture_output=True, text=True).stdout
+    orc = subprocess.run(["nm", "-D", "--defined-only", oracle.build()], capture_output=True, text=True).stdout
+    assert "orc_" not in prod
+    assert "dbuf_" not in orc
+
+
+def _plans_equal(r, c, k, m, A, cap=0):
+    st, off, s = oracle.plan(r, c, k, m, A, max_bucket=cap)
+    try:
+        p = rb.dbuf_plan(r, c, k, m, A, cap)
+    except rb.DbufError as e:
+        assert st != oracle.OK and e.status == rb.DBUF_EINFEASIBLE, (st, e)
+        return None
+    assert st == oracle.OK
+    info = rb.dbuf_plan_info(p)
+    assert info["slice"] == s, (r, c, k, m, A)
+    assert info["offsets"] == off.tolist(), (r, c, k, m, A)
+    assert info["bucket"] == s * m
+    assert info["padding"] == s * m - int(np.sum(np.asarray(r) * np.asarray(c)))
+    assert info["n_blocks"] == int(sum(-(-int(x) // int(y)) for x, y in zip(r, k)))
+    return info
+
+
+@pytest.mark.parametrize("name", [n for n in synth.WORKLOAD_NAMES])
+def test_planner_matches_oracle_on_workloads(name):
+    w = synth.workload(name)
+    r, c, k = w.arrays()
+    _plans_equal(r, c, k, w.m, w.align)
+
+
+def test_planner_matches_oracle_random():
+    rng = random.Random(2024)
+    for _ in range(3000):
+        n = rng.randint(1, 12)
+        rows = [rng.randint(1, 200) for _ in range(n)]
+        cols = [rng.choice([1, 2, 3, 7, 16, 48, 64]) for _ in range(n)]
+        k = [rng.randint(1, r) for r in rows]
+        m = rng.choice([1, 2, 3, 4, 8, 16, 64])
+        A = rng.choice([1, 2, 16, 32])
+        _plans_equal(rows, cols, k, m, A)
+
+
+def test_planner_matches_oracle_large_random():
+    """Buckets shaped like the stress workload, many m."""
+    rng = random.Random(77)
+    for _ in range(60):
+        n = rng.randint(5, 80)
+        rows = [int(np.exp(rng.uniform(np.log(64), np.log(16384)))) for _ in range(n)]
+        cols = [rng.choice(synth.workloads.STRESS_COLS) for _ in range(n)]
+        k = [min(rng.choice(synth.workloads.STRESS_KS), r) for r in rows]
+        _plans_equal(rows, cols, k, rng.choice([8, 64, 128, 1024]), 16)
+
+
+def test_planner_cap():
+    w = synth.workload("tiny_m4")
+    r, c, k = w.arrays()
+    assert _plans_equal(r, c, k, 4, 16, cap=147456) is not None
+    with pytest.raises(rb.DbufError) as e:
+        rb.dbuf_plan(r, c, k, 4, 16, 147455)
+    assert e.value.status == rb.DBUF_EINFEASIBLE
+
+
+@pytest.mark.parametrize("rows,cols,k,m,A", [
+    ([4], [4], [5], 2, 16),     # k > rows
+    ([0], [4], [1], 2, 16),     # rows < 1
+    ([4], [-1], [1], 2, 16),    # cols < 1
+    ([4], [4], [0], 2, 16),     # k < 1
+    ([4], [4], [1], 0, 16),     # m < 1
+    ([4], [4], [1], 2, 0),      # align < 1
+])
+def test_planner_rejects_invalid(rows, cols, k, m, A):
+    with pytest.raises(rb.DbufError) as e:
+        rb.dbuf_plan(rows, cols, k, m, A)
+    assert e.value.status == rb.DBUF_EINVAL
+    assert rb.dbuf_last_error()
+
+
+def test_empty_plan():
+    p = rb.dbuf_plan([], [], [], 8, 16)
+    info = rb.dbuf_plan_info(p)
+    assert info["slice"] == 0 and info["bucket"] == 0 and info["n_blocks"] == 0
+    assert rb.dbuf_required_bytes(p) > 0
+
+
+def test_required_bytes_cover_arrays():
+    for name in ("tiny_m4", "ragged_mix_m4", "llama_layer_m8"):
+        w = synth.workload(name)
+        r, c, k = w.arrays()
+        p = rb.dbuf_plan(r, c, k, w.m, 16)
+        info = rb.dbuf_plan_info(p)
+        need = rb.dbuf_required_bytes(p)
+        S, B = info["bucket"], info["n_blocks"]
+        assert need >= S * (4 + 2 + 2 + 1 + 1) + B * 8
+        assert need % 256 == 0
+        assert need < S * 10 + B * 8 + 64 * S // 100 + (1 << 20)
+
+
+def test_planner_time_budget():
+    """The pages report under 0.3 s of planning at init; time ours."""
+    import time
+    for name in ("moe_layer_m64", "ragged_stress_m8", "ragged_stress_m128", "ragged_stress_m1024"):
+        w = synth.workload(name)
+        r, c, k = w.arrays()
+        t = time.perf_counter()
+        rb.dbuf_plan(r, c, k, w.m, 16)
+        assert time.perf_counter() - t < 0.3
+
+
+@pytest.mark.parametrize("name", ["tiny_m4", "ragged_mix_m4", "ragged_mix_m8", "llama_layer_m8",
+                                  "moe_layer_m64", "ragged_stress_m8", "ragged_stress_m128"])
+def test_work_table_covers_bucket_once(name):
+    """Every element of the bucket is in exactly one work item; items respect
+    the kernel's limits; block numbers follow bucket order."""
+    w = synth.workload(name)
+    r, c, k = w.arrays()
+    p = rb.dbuf_plan(r, c, k, w.m, 16)
+    info = rb.dbuf_plan_info(p)
+    S = info["bucket"]
+    tab = rb.dbuf_work_table(p)
+    start, length = oracle.blocks(r, c, k, info["offsets"])   # bucket-order blocks
+    blk_of_start = {int(s): j for j, s in enumerate(start)}
+    cover = np.zeros(S + 1, np.int64)
+    seen_blocks = np.zeros(start.size, np.int64)
+    for t in tab:
+        e0, n = t["first_elem"], t["n_elems"]
+        assert 0 <= e0 and e0 + n <= S and n > 0
+        cover[e0] += 1
+        cover[e0 + n] -= 1
+        if t["kind"] == 2:
+            continue
+        j = blk_of_start[e0]                     # starts on a block edge
+        assert t["first_block"] == j
+        if t["kind"] == 0:
+            b = t["block_elems"]
+            assert 1 <= b <= 4096 and 1 <= t["n_blocks"] <= 256
+            assert (e0 % 16) + n <= 4096
+            assert np.all(length[j:j + t["n_blocks"] - 1] == b)
+            assert int(length[j:j + t["n_blocks"]].sum()) == n
+            seen_blocks[j:j + t["n_blocks"]] += 1
+        else:
+            assert t["kind"] == 1 and t["n_blocks"] == 1 and n == length[j]
+            seen_blocks[j] += 1
+    assert np.all(np.cumsum(cover)[:S] == 1)
+    assert np.all(seen_blocks == 1)
+    # padding items are exactly the padding
+    pad = oracle.padding_mask(r, c, info["offsets"], S)
+    zmask = np.zeros(S, bool)
+    for t in tab:
+        if t["kind"] == 2:
+            zmask[t["first_elem"]:t["first_elem"] + t["n_elems"]] = True
+    assert np.array_equal(zmask, pad)
