@@ -81,8 +81,11 @@ def test_copy_in_equals_zero_copy(name):
             oracle.pack(src, A.O.g[sl], 1.0 / w.m)
         A.O.step(hp_at(t), t, 1.0)
         ga, gb = A.gpu_state(), B.gpu_state()
-        for key in ga:
+        for key in ("p", "pb", "mq", "vq", "sc"):   # the grad buckets hold g/m and g
             assert np.array_equal(ga[key].view(np.uint8), gb[key].view(np.uint8)), key
+        gb_scaled = np.zeros_like(gb["g"])
+        oracle.pack(gb["g"], gb_scaled, 1.0 / w.m)
+        assert np.array_equal(ga["g"], gb_scaled)
         compare(ga, A.oracle_state(), A.O.pad)
     assert A.D.device_status() == 0
 
