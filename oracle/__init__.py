@@ -159,7 +159,8 @@ def padding_mask(rows, cols, offsets, bucket):
 # ---------------------------------------------------------------- update ---
 
 def step_scalars(lr, beta1, beta2, eps, wd, t):
-    """(b1, 1-b1, b2, 1-b2, sqrt(1-b2^t), eps, lr/(1-b1^t), 1-lr*wd) as float32."""
+    """(b1, 1-b1, b2, 1-b2, sqrt(1-b2^t), eps*sqrt(1-b2^t), lr*sqrt(1-b2^t)/(1-b1^t),
+    1-lr*wd) as float32."""
     out = np.zeros(8, dtype=np.float32)
     _load().orc_step_scalars(lr, beta1, beta2, eps, wd, int(t), out.ctypes.data)
     return out

@@ -272,22 +272,28 @@ static float bf16_to_f32(uint16_t h) {
 
 // Per-step scalars of Adam with bias correction and decoupled weight decay,
 // formed in double from the float hyper-parameters, rounded to float once.
+// The bias corrections are folded into the step size and eps, as the
+// published 8-bit optimizers do (Dettmers et al., "8-bit Optimizers via
+// Block-wise Quantization", ICLR 2022):
+//   (lr / bc1) * m / (sqrt(v) / sqrt(bc2) + eps)
+//     = (lr * sqrt(bc2) / bc1) * m / (sqrt(v) + eps * sqrt(bc2)),
+// with bc1 = 1 - b1^t, bc2 = 1 - b2^t: one division per element.
 struct Scalars {
-    float b1, omb1, b2, omb2, bc2s, eps, step, decay;
+    float b1, omb1, b2, omb2, sqrt_bc2, eps_hat, step_hat, decay;
 };
 
 static Scalars make_scalars(float lr, float beta1, float beta2, float eps, float wd, int64_t t) {
-    double l = lr, B1 = beta1, B2 = beta2, W = wd;
+    double l = lr, B1 = beta1, B2 = beta2, E = eps, W = wd;
     double bc1 = 1.0 - std::pow(B1, (double)t);
-    double bc2 = 1.0 - std::pow(B2, (double)t);
+    double sq2 = std::sqrt(1.0 - std::pow(B2, (double)t));
     Scalars c;
     c.b1 = (float)B1;
     c.omb1 = (float)(1.0 - B1);
     c.b2 = (float)B2;
     c.omb2 = (float)(1.0 - B2);
-    c.bc2s = (float)std::sqrt(bc2);
-    c.eps = eps;
-    c.step = (float)(l / bc1);
+    c.sqrt_bc2 = (float)sq2;
+    c.eps_hat = (float)(E * sq2);
+    c.step_hat = (float)(l * sq2 / bc1);
     c.decay = (float)(1.0 - l * W);
     return c;
 }
@@ -320,11 +326,10 @@ static void adam8_block(int64_t len, float* p, const uint16_t* g, int8_t* mq, ui
         t = c.omb2 * gg;
         v = v + t;
         float r = std::sqrt(v);
-        float d = r / c.bc2s;
-        d = d + c.eps;
+        float d = r + c.eps_hat;
         float u = m / d;
         float pn = p[i] * c.decay;
-        t = c.step * u;
+        t = c.step_hat * u;
         pn = pn - t;
         p[i] = pn;
         pb[i] = bf16_rne(pn);
@@ -371,11 +376,11 @@ void orc_adam8_step(int64_t n_blocks, const int64_t* start, const int64_t* len, 
     }
 }
 
-// The per-step scalars as floats, in the order b1, omb1, b2, omb2, bc2s, eps,
-// step, decay (for the tests' closed forms).
+// The per-step scalars as floats, in the order b1, omb1, b2, omb2, sqrt_bc2,
+// eps_hat, step_hat, decay (for the tests' closed forms).
 void orc_step_scalars(float lr, float beta1, float beta2, float eps, float wd, int64_t t, float* out) {
     Scalars c = make_scalars(lr, beta1, beta2, eps, wd, t);
-    float v[8] = {c.b1, c.omb1, c.b2, c.omb2, c.bc2s, c.eps, c.step, c.decay};
+    float v[8] = {c.b1, c.omb1, c.b2, c.omb2, c.sqrt_bc2, c.eps_hat, c.step_hat, c.decay};
     std::memcpy(out, v, sizeof v);
 }
 

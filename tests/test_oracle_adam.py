@@ -230,13 +230,13 @@ def test_threads_do_not_change_results():
 
 def test_step_scalars_closed_forms():
     c = oracle.step_scalars(1e-3, 0.9, 0.999, 1e-8, 0.01, 3)
-    b1, omb1, b2, omb2, bc2s, eps, step, decay = [float(x) for x in c]
-    B1, B2, lr, wd = f32(0.9), f32(0.999), f32(1e-3), f32(0.01)
+    b1, omb1, b2, omb2, sq2, eps_hat, step_hat, decay = [float(x) for x in c]
+    B1, B2, lr, wd, eps = f32(0.9), f32(0.999), f32(1e-3), f32(0.01), f32(1e-8)
     assert b1 == f32(B1) and omb1 == f32(1 - B1) and b2 == f32(B2) and omb2 == f32(1 - B2)
-    assert bc2s == f32(np.sqrt(1 - B2 ** 3))
-    assert step == f32(lr / (1 - B1 ** 3))
+    assert sq2 == f32(np.sqrt(1 - B2 ** 3))
+    assert eps_hat == f32(eps * np.sqrt(1 - B2 ** 3))
+    assert step_hat == f32(lr * np.sqrt(1 - B2 ** 3) / (1 - B1 ** 3))
     assert decay == f32(1 - lr * wd)
-    assert eps == f32(1e-8)
 
 
 def test_bf16_rounding_matches_torch():

@@ -21,10 +21,11 @@ MUTANTS = {
                "test_oracle_adam.py::test_golden_first_step"),
     "no_decay": ("        float pn = p[i] * c.decay;", "        float pn = p[i];",
                  "test_oracle_adam.py::test_golden_first_step"),
-    "no_bias_corr2": ("        float d = r / c.bc2s;", "        float d = r;",
-                      "test_oracle_adam.py::test_golden_first_step"),
-    "eps_inside_sqrt": ("        float r = std::sqrt(v);\n        float d = r / c.bc2s;\n        d = d + c.eps;",
-                        "        float r = std::sqrt(v);\n        float d = std::sqrt(v + c.eps) / c.bc2s;",
+    "no_bias_corr2_step": ("    c.step_hat = (float)(l * sq2 / bc1);", "    c.step_hat = (float)(l / bc1);",
+                           "test_oracle_adam.py::test_golden_first_step"),
+    "no_bias_corr2_eps": ("    c.eps_hat = (float)(E * sq2);", "    c.eps_hat = (float)(E);",
+                          "test_oracle_adam.py::test_first_step_closed_form"),
+    "eps_inside_sqrt": ("        float d = r + c.eps_hat;", "        float d = std::sqrt(v + c.eps_hat);",
                         "test_oracle_adam.py::test_first_step_closed_form"),
     "m_dequant_255": ("    const float dqm = *sm / 127.0f;", "    const float dqm = *sm / 255.0f;",
                       "test_oracle_adam.py::test_uniform_magnitude_blocks_reduce_to_adamw"),
@@ -37,7 +38,7 @@ MUTANTS = {
                       "test_oracle_adam.py::test_uniform_magnitude_blocks_reduce_to_adamw"),
     "beta_swap": ("        float m = c.b1 * mo;", "        float m = c.b2 * mo;",
                   "test_oracle_adam.py::test_uniform_magnitude_blocks_reduce_to_adamw"),
-    "no_bias_corr1": ("    c.step = (float)(l / bc1);", "    c.step = (float)(l);",
+    "no_bias_corr1": ("    c.step_hat = (float)(l * sq2 / bc1);", "    c.step_hat = (float)(l * sq2);",
                       "test_oracle_adam.py::test_first_step_closed_form"),
     "coupled_decay": ("        float gi = bf16_to_f32(g[i]) * grad_scale;",
                       "        float gi = bf16_to_f32(g[i]) * grad_scale + 0.01f * p[i];",
