@@ -122,8 +122,10 @@ typedef struct {
  * (fp32, each operation rounded separately, in this order):
  *   g = grad * grad_scale;  m_old = qm * scale_m / 127;  s = qv * scale_v / 255;
  *   m = b1*m_old + (1-b1)*g;  v = b2*s*s + (1-b2)*g*g;  r = sqrt(v);
- *   p = p*(1 - lr*wd) - (lr/(1-b1^t)) * m / (r/sqrt(1-b2^t) + eps);
+ *   p = p*(1 - lr*wd) - step_hat * m / (r + eps_hat);
  *   param_bf16 = round-to-nearest-even(p)
+ * with the bias corrections folded into step_hat = lr*sqrt(1-b2^t)/(1-b1^t)
+ * and eps_hat = eps*sqrt(1-b2^t) (the same Adam step in exact arithmetic);
  * per block: scale_m = max|m|, scale_v = max r, qm = rint(m*127/scale_m)
  * clamped to [-127,127], qv = rint(r*255/scale_v) clamped to [0,255] (codes
  * 0 where the scale is 0).  Per-step scalars are formed in double, rounded to

@@ -58,9 +58,9 @@ extern "C" const char* dbuf_last_error(void) { return dbuf_detail::g_err.c_str()
 
 namespace {
 
-constexpr int kThreads = 256;          // threads per CTA of the step kernel
-constexpr int kVec = 16;               // elements per thread-vector
-constexpr int kTile = kThreads * kVec; // 4096 elements per tile
+constexpr int kThreads = 512;          // threads per CTA of the step kernel
+constexpr int kAlign = 16;             // tensor starts are multiples of 16 elements
+constexpr int kTile = 4096;            // elements per tile (8 per thread)
 constexpr int kMaxBlk = 256;           // blocks per WHOLE tile
 constexpr int64_t kZeroChunk = 65536;  // elements per ZERO tile
 constexpr int64_t kPackChunk = 16384;  // elements per copy-in CTA (32 KB)
@@ -110,7 +110,7 @@ void build_tiles(const dbuf_plan_s& p, std::vector<Tile>& tiles) {
         while (j < nb) {
             const int64_t e0 = o + j * b;
             if (b <= kTile) {
-                const int64_t cap = kTile - (e0 & (kVec - 1));
+                const int64_t cap = kTile - (e0 & (kAlign - 1));
                 const int64_t q = std::min<int64_t>({kMaxBlk, cap / b, nb - j});
                 if (q >= 1) {
                     whole.push_back(Tile{e0, blk + j, std::min(q * b, n - j * b), (int32_t)b, TILE_WHOLE,
@@ -195,156 +195,266 @@ struct dbuf_s {
 
 namespace {
 
+// Per-step scalars (formed on the host in double, rounded to float once).
+// The bias corrections are folded into the step size and eps:
+//   (lr/bc1) m / (sqrt(v)/sqrt(bc2) + eps) = step_hat * m / (sqrt(v) + eps_hat).
 struct StepC {
-    float b1, omb1, b2, omb2, bc2s, eps, step, decay, gscale;
+    float b1, omb1, b2, omb2, eps_hat, step_hat, decay, gscale;
 };
 
-__device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) { return __uint_as_float(h << 16); }
+constexpr int kV = 8;  // elements per thread-vector in the step kernel
 
 __device__ __forceinline__ void set_status(int32_t* status, int32_t code) { atomicCAS(status, 0, code); }
 
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) { return __uint_as_float(h << 16); }
+
+// Code bytes to float without the conversion unit: a byte b placed in the
+// low mantissa bits of 2^23 reads as 2^23 + b; subtracting 2^23 is exact.
+// int8 codes are stored with the sign bit flipped first (b = code + 128).
+__device__ __forceinline__ float ubyte_to_f(uint32_t w, uint32_t sel) {
+    return __fsub_rn(__uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540u | sel)), 8388608.0f);
+}
+__device__ __forceinline__ float sbyte_to_f(uint32_t w_flipped, uint32_t sel) {
+    return __fsub_rn(__uint_as_float(__byte_perm(w_flipped, 0x4B000000u, 0x7540u | sel)), 8388736.0f);
+}
+
+// Round to the nearest integer, ties to even, by adding 1.5*2^23: the sum
+// lies where the float spacing is 1, so the addition itself rounds; the
+// low byte of the result's bits is the integer's two's-complement low byte.
+// Valid for |x| < 2^22; the codes here satisfy |x| <= 255.
+__device__ __forceinline__ uint32_t rne_low_bits(float x) { return __float_as_uint(__fadd_rn(x, 12582912.0f)); }
+
+__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    return __byte_perm(__byte_perm(a, b, 0x0040u), __byte_perm(c, d, 0x0040u), 0x5410u);
+}
+
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
 // New m and sqrt(v) of one element, every operation rounded on its own.
-__device__ __forceinline__ void new_m_r(float graw, float qm, float qv, float dqm, float dqv,
-                                        const StepC& c, float& m, float& r) {
+__device__ __forceinline__ void new_m_r(float graw, float qmf, float qvf, float dqm, float dqv, const StepC& c,
+                                        float& m, float& r) {
     const float g = __fmul_rn(graw, c.gscale);
-    const float mo = __fmul_rn(qm, dqm);
-    const float so = __fmul_rn(qv, dqv);
+    const float mo = __fmul_rn(qmf, dqm);
+    const float so = __fmul_rn(qvf, dqv);
     const float vo = __fmul_rn(so, so);
     m = __fadd_rn(__fmul_rn(c.b1, mo), __fmul_rn(c.omb1, g));
-    const float gg = __fmul_rn(g, g);
-    const float v = __fadd_rn(__fmul_rn(c.b2, vo), __fmul_rn(c.omb2, gg));
+    const float v = __fadd_rn(__fmul_rn(c.b2, vo), __fmul_rn(c.omb2, __fmul_rn(g, g)));
     r = __fsqrt_rn(v);
 }
 
 __device__ __forceinline__ float new_p(float p, float m, float r, const StepC& c) {
-    const float d = __fadd_rn(__fdiv_rn(r, c.bc2s), c.eps);
-    const float u = __fdiv_rn(m, d);
-    return __fsub_rn(__fmul_rn(p, c.decay), __fmul_rn(c.step, u));
+    const float u = __fdiv_rn(m, __fadd_rn(r, c.eps_hat));
+    return __fsub_rn(__fmul_rn(p, c.decay), __fmul_rn(c.step_hat, u));
 }
 
-__device__ __forceinline__ uint32_t code_m(float m, float q) {
-    float a = rintf(__fmul_rn(m, q));
-    a = fminf(127.f, fmaxf(-127.f, a));
-    return (uint32_t)((int32_t)a) & 0xffu;
-}
-
-__device__ __forceinline__ uint32_t code_v(float r, float q) {
-    float b = rintf(__fmul_rn(r, q));
-    b = fminf(255.f, fmaxf(0.f, b));
-    return (uint32_t)b;
-}
-
-// Registers of one thread-vector: 16 consecutive bucket elements.
-struct Vec16 {
-    uint32_t g[8];   // bf16 pairs
-    float p[16];
-    uint32_t mq[4];  // 16 int8 codes
-    uint32_t vq[4];  // 16 uint8 codes
+// Inputs of one thread-vector (8 consecutive bucket elements).
+struct In8 {
+    uint32_t g[4];   // bf16 pairs
+    float p[8];
+    uint32_t mq[2];  // int8 codes with the sign bit flipped
+    uint32_t vq[2];  // uint8 codes
 };
 
-__device__ __forceinline__ uint32_t byte_of(const uint32_t* w, int i) { return (w[i >> 2] >> (8 * (i & 3))) & 0xffu; }
-__device__ __forceinline__ float gval(const uint32_t* g, int i) { return bf16_bits_to_f32((g[i >> 1] >> (16 * (i & 1))) & 0xffffu); }
-
-// Load elements [vb, vb+16) clipped to [lo, hi); out-of-range lanes read 0.
-__device__ __forceinline__ void load_vec(Vec16& x, int64_t vb, int64_t lo, int64_t hi, bool full, bool want_p,
-                                         const float* master, const uint16_t* grad, const int8_t* mq,
-                                         const uint8_t* vq) {
-    if (full) {
-        const uint4 g0 = __ldg(reinterpret_cast<const uint4*>(grad + vb));
-        const uint4 g1 = __ldg(reinterpret_cast<const uint4*>(grad + vb) + 1);
-        x.g[0] = g0.x; x.g[1] = g0.y; x.g[2] = g0.z; x.g[3] = g0.w;
-        x.g[4] = g1.x; x.g[5] = g1.y; x.g[6] = g1.z; x.g[7] = g1.w;
-        const uint4 a = *reinterpret_cast<const uint4*>(mq + vb);
-        const uint4 b = *reinterpret_cast<const uint4*>(vq + vb);
-        x.mq[0] = a.x; x.mq[1] = a.y; x.mq[2] = a.z; x.mq[3] = a.w;
-        x.vq[0] = b.x; x.vq[1] = b.y; x.vq[2] = b.z; x.vq[3] = b.w;
+// Load elements [vb, vb+8); when !FULL only those in [lo, hi) are read and
+// the rest are zero.
+template <bool FULL>
+__device__ __forceinline__ void load8(In8& x, int64_t vb, int64_t lo, int64_t hi, bool want_p, const float* master,
+                                      const uint16_t* grad, const int8_t* mq, const uint8_t* vq) {
+    if (FULL) {
+        const uint4 g = __ldg(reinterpret_cast<const uint4*>(grad + vb));
+        x.g[0] = g.x; x.g[1] = g.y; x.g[2] = g.z; x.g[3] = g.w;
+        const uint2 a = *reinterpret_cast<const uint2*>(mq + vb);
+        const uint2 b = *reinterpret_cast<const uint2*>(vq + vb);
+        x.mq[0] = a.x ^ 0x80808080u; x.mq[1] = a.y ^ 0x80808080u;
+        x.vq[0] = b.x; x.vq[1] = b.y;
         if (want_p) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float4 f = __ldcs(reinterpret_cast<const float4*>(master + vb) + q);
-                x.p[4 * q] = f.x; x.p[4 * q + 1] = f.y; x.p[4 * q + 2] = f.z; x.p[4 * q + 3] = f.w;
-            }
+            const float4 p0 = __ldcs(reinterpret_cast<const float4*>(master + vb));
+            const float4 p1 = __ldcs(reinterpret_cast<const float4*>(master + vb) + 1);
+            x.p[0] = p0.x; x.p[1] = p0.y; x.p[2] = p0.z; x.p[3] = p0.w;
+            x.p[4] = p1.x; x.p[5] = p1.y; x.p[6] = p1.z; x.p[7] = p1.w;
         }
     } else {
+        uint32_t g[4] = {0, 0, 0, 0}, a[2] = {0, 0}, b[2] = {0, 0};
 #pragma unroll
-        for (int i = 0; i < 8; ++i) x.g[i] = 0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) x.mq[i] = x.vq[i] = 0;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
+        for (int i = 0; i < kV; ++i) {
             const int64_t e = vb + i;
             const bool in = (e >= lo && e < hi);
             x.p[i] = (in && want_p) ? master[e] : 0.f;
             if (in) {
-                x.g[i >> 1] |= (uint32_t)grad[e] << (16 * (i & 1));
-                x.mq[i >> 2] |= ((uint32_t)(uint8_t)mq[e]) << (8 * (i & 3));
-                x.vq[i >> 2] |= ((uint32_t)vq[e]) << (8 * (i & 3));
+                g[i >> 1] |= (uint32_t)grad[e] << (16 * (i & 1));
+                a[i >> 2] |= (uint32_t)(uint8_t)mq[e] << (8 * (i & 3));
+                b[i >> 2] |= (uint32_t)vq[e] << (8 * (i & 3));
             }
         }
+        x.g[0] = g[0]; x.g[1] = g[1]; x.g[2] = g[2]; x.g[3] = g[3];
+        x.mq[0] = a[0] ^ 0x80808080u; x.mq[1] = a[1] ^ 0x80808080u;
+        x.vq[0] = b[0]; x.vq[1] = b[1];
     }
 }
 
-__device__ __forceinline__ void store_p_bf16(const float* p, int64_t vb, int64_t lo, int64_t hi, bool full,
-                                             float* master, uint16_t* param) {
-    uint32_t h[8];
+__device__ __forceinline__ float g_of(const In8& x, int i) {
+    const uint32_t w = x.g[i >> 1];
+    return __uint_as_float((i & 1) ? (w & 0xffff0000u) : (w << 16));
+}
+
+// Update 8 elements; dq* are per element (equal when the vector lies in one block).
+__device__ __forceinline__ void update8(In8& x, const float* dqm, const float* dqv, const StepC& c, float* m,
+                                        float* r) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const uint32_t a = __bfloat16_as_ushort(__float2bfloat16_rn(p[2 * i]));
-        const uint32_t b = __bfloat16_as_ushort(__float2bfloat16_rn(p[2 * i + 1]));
-        h[i] = a | (b << 16);
+    for (int i = 0; i < kV; ++i) {
+        new_m_r(g_of(x, i), sbyte_to_f(x.mq[i >> 2], i & 3), ubyte_to_f(x.vq[i >> 2], i & 3), dqm[i], dqv[i], c, m[i],
+                r[i]);
+        x.p[i] = new_p(x.p[i], m[i], r[i], c);
     }
-    if (full) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-            __stcs(reinterpret_cast<float4*>(master + vb) + q,
-                   make_float4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]));
-        __stcs(reinterpret_cast<uint4*>(param + vb), make_uint4(h[0], h[1], h[2], h[3]));
-        __stcs(reinterpret_cast<uint4*>(param + vb) + 1, make_uint4(h[4], h[5], h[6], h[7]));
+}
+
+template <bool FULL>
+__device__ __forceinline__ void store_p8(const float* p, int64_t vb, int64_t lo, int64_t hi, float* master,
+                                         uint16_t* param) {
+    const uint4 h = make_uint4(bf16x2_bits(p[0], p[1]), bf16x2_bits(p[2], p[3]), bf16x2_bits(p[4], p[5]),
+                               bf16x2_bits(p[6], p[7]));
+    if (FULL) {
+        __stcs(reinterpret_cast<float4*>(master + vb), make_float4(p[0], p[1], p[2], p[3]));
+        __stcs(reinterpret_cast<float4*>(master + vb) + 1, make_float4(p[4], p[5], p[6], p[7]));
+        __stcs(reinterpret_cast<uint4*>(param + vb), h);
     } else {
+        const uint32_t hw[4] = {h.x, h.y, h.z, h.w};
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
+        for (int i = 0; i < kV; ++i) {
             const int64_t e = vb + i;
             if (e >= lo && e < hi) {
                 master[e] = p[i];
-                param[e] = (uint16_t)((h[i >> 1] >> (16 * (i & 1))) & 0xffffu);
+                param[e] = (uint16_t)(hw[i >> 1] >> (16 * (i & 1)));
             }
         }
     }
 }
 
-__device__ __forceinline__ void store_codes(const uint32_t* cm, const uint32_t* cv, int64_t vb, int64_t lo,
-                                            int64_t hi, bool full, int8_t* mq, uint8_t* vq) {
-    if (full) {
-        __stcs(reinterpret_cast<uint4*>(mq + vb), make_uint4(cm[0], cm[1], cm[2], cm[3]));
-        __stcs(reinterpret_cast<uint4*>(vq + vb), make_uint4(cv[0], cv[1], cv[2], cv[3]));
+// Codes of 8 elements from m, r and the per-element quotients 127/absmax,
+// 255/absmax.  |m*qm| <= 127 and 0 <= r*qv <= 255 hold by construction
+// (absmax over the same values), so rounding never needs a clamp.
+template <bool FULL>
+__device__ __forceinline__ void store_codes8(const float* m, const float* r, const float* qm, const float* qv,
+                                             int64_t vb, int64_t lo, int64_t hi, int8_t* mq, uint8_t* vq) {
+    uint32_t bm[kV], bv[kV];
+#pragma unroll
+    for (int i = 0; i < kV; ++i) {
+        bm[i] = rne_low_bits(__fmul_rn(m[i], qm[i]));
+        bv[i] = rne_low_bits(__fmul_rn(r[i], qv[i]));
+    }
+    const uint2 cm = make_uint2(pack_low_bytes(bm[0], bm[1], bm[2], bm[3]), pack_low_bytes(bm[4], bm[5], bm[6], bm[7]));
+    const uint2 cv = make_uint2(pack_low_bytes(bv[0], bv[1], bv[2], bv[3]), pack_low_bytes(bv[4], bv[5], bv[6], bv[7]));
+    if (FULL) {
+        __stcs(reinterpret_cast<uint2*>(mq + vb), cm);
+        __stcs(reinterpret_cast<uint2*>(vq + vb), cv);
     } else {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
+        for (int i = 0; i < kV; ++i) {
             const int64_t e = vb + i;
             if (e >= lo && e < hi) {
-                mq[e] = (int8_t)byte_of(cm, i);
-                vq[e] = (uint8_t)byte_of(cv, i);
+                mq[e] = (int8_t)(bm[i] & 0xffu);
+                vq[e] = (uint8_t)(bv[i] & 0xffu);
             }
         }
     }
 }
 
 // Max over the lanes of a warp that share `key`, where lanes with equal keys
-// are contiguous; the first lane of each run gets the run's maximum.
-__device__ __forceinline__ void segmented_max(int key, uint32_t& a, uint32_t& b, bool& head) {
+// are contiguous; the first lane of each run ends with the run's maximum.
+__device__ __forceinline__ bool segmented_max(int key, float& a, float& b) {
     const int lane = threadIdx.x & 31;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
         const int ok = __shfl_down_sync(0xffffffffu, key, d);
-        const uint32_t oa = __shfl_down_sync(0xffffffffu, a, d);
-        const uint32_t ob = __shfl_down_sync(0xffffffffu, b, d);
+        const float oa = __shfl_down_sync(0xffffffffu, a, d);
+        const float ob = __shfl_down_sync(0xffffffffu, b, d);
         if (lane + d < 32 && ok == key) {
-            a = max(a, oa);
-            b = max(b, ob);
+            a = fmaxf(a, oa);
+            b = fmaxf(b, ob);
         }
     }
     const int prev = __shfl_up_sync(0xffffffffu, key, 1);
-    head = (lane == 0) || (prev != key);
+    return (lane == 0) || (prev != key);
+}
+
+__device__ __forceinline__ void warp_max2(float& a, float& b) {
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) {
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, d));
+        b = fmaxf(b, __shfl_xor_sync(0xffffffffu, b, d));
+    }
+}
+
+// Non-negative floats order like their bit patterns, so the block maxima
+// are kept as unsigned integers for atomicMax in shared memory.
+template <bool FULL>
+__device__ __forceinline__ void whole_vec(const Tile& t, int64_t vb, int64_t lo, int64_t hi, bool multi,
+                                          float* master, uint16_t* param, const uint16_t* grad, int8_t* mq,
+                                          uint8_t* vq, const StepC& c, const float* s_dqm, const float* s_dqv,
+                                          const float* s_qm, const float* s_qv, uint32_t* s_am, uint32_t* s_ar) {
+    const int tid = threadIdx.x;
+    const int64_t elo = max(vb, lo), ehi = min(vb + kV, hi);
+    const bool any = elo < ehi;
+    const uint32_t b = (uint32_t)t.b;
+    // block of each element (all equal unless blocks are shorter than a vector
+    // or start off the 8-element grid)
+    const int bf = any ? (multi ? (int)((uint32_t)(elo - lo) / b) : 0) : -1;
+    const int bl = any ? (multi ? (int)((uint32_t)(ehi - 1 - lo) / b) : 0) : -1;
+    const bool one = (bf == bl);
+    int blk[kV];
+    float dqm[kV], dqv[kV], m[kV], r[kV];
+    In8 x;
+    if (any) {
+        load8<FULL>(x, vb, lo, hi, true, master, grad, mq, vq);
+#pragma unroll
+        for (int i = 0; i < kV; ++i) {
+            const int64_t e = vb + i;
+            blk[i] = (one || e < lo || e >= hi) ? bf : (int)((uint32_t)(e - lo) / b);
+            dqm[i] = s_dqm[blk[i]];
+            dqv[i] = s_dqv[blk[i]];
+        }
+        update8(x, dqm, dqv, c, m, r);
+        store_p8<FULL>(x.p, vb, lo, hi, master, param);
+    }
+    // absmax per block (elements outside the tile have m = r = 0)
+    float am = 0.f, ar = 0.f;
+    if (any && one) {
+#pragma unroll
+        for (int i = 0; i < kV; ++i) {
+            am = fmaxf(am, fabsf(m[i]));
+            ar = fmaxf(ar, r[i]);
+        }
+    } else if (any) {
+#pragma unroll
+        for (int i = 0; i < kV; ++i) {
+            atomicMax(&s_am[blk[i]], __float_as_uint(fabsf(m[i])));
+            atomicMax(&s_ar[blk[i]], __float_as_uint(r[i]));
+        }
+    }
+    const int key = (any && one) ? bf : -1;
+    if (segmented_max(key, am, ar) && key >= 0) {
+        atomicMax(&s_am[key], __float_as_uint(am));
+        atomicMax(&s_ar[key], __float_as_uint(ar));
+    }
+    __syncthreads();
+    if (tid < t.nblk) {
+        const float AMm = __uint_as_float(s_am[tid]), AMr = __uint_as_float(s_ar[tid]);
+        const_cast<float*>(s_qm)[tid] = AMm > 0.f ? __fdiv_rn(127.f, AMm) : 0.f;
+        const_cast<float*>(s_qv)[tid] = AMr > 0.f ? __fdiv_rn(255.f, AMr) : 0.f;
+    }
+    __syncthreads();
+    if (any) {
+        float qm[kV], qv[kV];
+#pragma unroll
+        for (int i = 0; i < kV; ++i) {
+            qm[i] = s_qm[blk[i]];
+            qv[i] = s_qv[blk[i]];
+        }
+        store_codes8<FULL>(m, r, qm, qv, vb, lo, hi, mq, vq);
+    }
 }
 
 __device__ void whole_tile(const Tile& t, float* master, uint16_t* param, const uint16_t* grad, int8_t* mq,
@@ -360,182 +470,116 @@ __device__ void whole_tile(const Tile& t, float* master, uint16_t* param, const 
         s_ar[tid] = 0u;
     }
     __syncthreads();
-
     const int64_t lo = t.e0, hi = t.e0 + t.n;
-    const int64_t vb = (t.e0 & ~int64_t(kVec - 1)) + (int64_t)kVec * tid;
-    const int64_t elo = max(vb, lo), ehi = min(vb + kVec, hi);
-    const bool any = elo < ehi;
-    const bool full = (elo == vb) && (ehi == vb + kVec);
-    const int32_t b = t.b;
+    const int64_t vb = (t.e0 & ~int64_t(kAlign - 1)) + (int64_t)kV * tid;
+    const bool full = (vb >= lo) && (vb + kV <= hi);
+    const bool multi = t.nblk > 1;
+    if (full)
+        whole_vec<true>(t, vb, lo, hi, multi, master, param, grad, mq, vq, c, s_dqm, s_dqv, s_qm, s_qv, s_am, s_ar);
+    else
+        whole_vec<false>(t, vb, lo, hi, multi, master, param, grad, mq, vq, c, s_dqm, s_dqv, s_qm, s_qv, s_am, s_ar);
+    if (tid < t.nblk) scales[t.blk0 + tid] = make_float2(__uint_as_float(s_am[tid]), __uint_as_float(s_ar[tid]));
+}
 
-    Vec16 x;
-    float m[16], r[16];
-    int blk_first = -1, blk_last = -1;
-    if (any) {
-        load_vec(x, vb, lo, hi, full, true, master, grad, mq, vq);
-        blk_first = (int)((elo - lo) / b);
-        blk_last = (int)((ehi - 1 - lo) / b);
-        const bool one = (blk_first == blk_last);
-        const float dqm1 = s_dqm[blk_first], dqv1 = s_dqv[blk_first];
+template <bool FULL>
+__device__ __forceinline__ void large_pass1_vec(int64_t vb, int64_t lo, int64_t hi, float dqm1, float dqv1,
+                                                float* master, uint16_t* param, const uint16_t* grad,
+                                                const int8_t* mq, const uint8_t* vq, const StepC& c, float& am,
+                                                float& ar) {
+    In8 x;
+    float dqm[kV], dqv[kV], m[kV], r[kV];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            float dqm = dqm1, dqv = dqv1;
-            if (!one) {
-                const int64_t e = vb + i;
-                const int lb = (e >= lo && e < hi) ? (int)((e - lo) / b) : blk_first;
-                dqm = s_dqm[lb];
-                dqv = s_dqv[lb];
-            }
-            new_m_r(gval(x.g, i), (float)(int8_t)byte_of(x.mq, i), (float)byte_of(x.vq, i), dqm, dqv, c, m[i], r[i]);
-            x.p[i] = new_p(x.p[i], m[i], r[i], c);
-        }
-        store_p_bf16(x.p, vb, lo, hi, full, master, param);
+    for (int i = 0; i < kV; ++i) {
+        dqm[i] = dqm1;
+        dqv[i] = dqv1;
     }
+    load8<FULL>(x, vb, lo, hi, true, master, grad, mq, vq);
+    update8(x, dqm, dqv, c, m, r);
+    store_p8<FULL>(x.p, vb, lo, hi, master, param);
+#pragma unroll
+    for (int i = 0; i < kV; ++i) {
+        am = fmaxf(am, fabsf(m[i]));
+        ar = fmaxf(ar, r[i]);
+    }
+}
 
-    // Per-block absmax of |m| and r (non-negative floats compare as integers).
-    const bool one = any && (blk_first == blk_last);
-    uint32_t am = 0u, ar = 0u;
-    if (one) {
+template <bool FULL>
+__device__ __forceinline__ void large_pass2_vec(int64_t vb, int64_t lo, int64_t hi, float dqm1, float dqv1,
+                                                float qm1, float qv1, const uint16_t* grad, int8_t* mq, uint8_t* vq,
+                                                const StepC& c) {
+    In8 x;
+    float m[kV], r[kV], qm[kV], qv[kV];
+    load8<FULL>(x, vb, lo, hi, false, nullptr, grad, mq, vq);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int64_t e = vb + i;
-            if (full || (e >= lo && e < hi)) {
-                am = max(am, __float_as_uint(fabsf(m[i])));
-                ar = max(ar, __float_as_uint(r[i]));
-            }
-        }
-    } else if (any) {
-        for (int i = 0; i < 16; ++i) {
-            const int64_t e = vb + i;
-            if (e >= lo && e < hi) {
-                const int lb = (int)((e - lo) / b);
-                atomicMax(&s_am[lb], __float_as_uint(fabsf(m[i])));
-                atomicMax(&s_ar[lb], __float_as_uint(r[i]));
-            }
-        }
+    for (int i = 0; i < kV; ++i) {
+        new_m_r(g_of(x, i), sbyte_to_f(x.mq[i >> 2], i & 3), ubyte_to_f(x.vq[i >> 2], i & 3), dqm1, dqv1, c, m[i],
+                r[i]);
+        qm[i] = qm1;
+        qv[i] = qv1;
     }
-    bool head;
-    const int key = one ? blk_first : -1;
-    segmented_max(key, am, ar, head);
-    if (one && head) {
-        atomicMax(&s_am[key], am);
-        atomicMax(&s_ar[key], ar);
-    }
-    __syncthreads();
-    if (tid < t.nblk) {
-        const float AMm = __uint_as_float(s_am[tid]), AMr = __uint_as_float(s_ar[tid]);
-        s_qm[tid] = AMm > 0.f ? __fdiv_rn(127.f, AMm) : 0.f;
-        s_qv[tid] = AMr > 0.f ? __fdiv_rn(255.f, AMr) : 0.f;
-        scales[t.blk0 + tid] = make_float2(AMm, AMr);
-    }
-    __syncthreads();
-    if (any) {
-        uint32_t cm[4] = {0, 0, 0, 0}, cv[4] = {0, 0, 0, 0};
-        const float qm1 = s_qm[blk_first], qv1 = s_qv[blk_first];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            float qm = qm1, qv = qv1;
-            if (!one) {
-                const int64_t e = vb + i;
-                const int lb = (e >= lo && e < hi) ? (int)((e - lo) / b) : blk_first;
-                qm = s_qm[lb];
-                qv = s_qv[lb];
-            }
-            cm[i >> 2] |= code_m(m[i], qm) << (8 * (i & 3));
-            cv[i >> 2] |= code_v(r[i], qv) << (8 * (i & 3));
-        }
-        store_codes(cm, cv, vb, lo, hi, full, mq, vq);
-    }
+    store_codes8<FULL>(m, r, qm, qv, vb, lo, hi, mq, vq);
 }
 
 __device__ void large_block(const Tile& t, float* master, uint16_t* param, const uint16_t* grad, int8_t* mq,
                             uint8_t* vq, float2* scales, const StepC& c) {
-    __shared__ uint32_t s_red[2][kThreads / 32];
+    __shared__ float s_red[2][kThreads / 32];
     __shared__ float s_q[2];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const float2 sc = scales[t.blk0];
     const float dqm = __fdiv_rn(sc.x, 127.f), dqv = __fdiv_rn(sc.y, 255.f);
     const int64_t lo = t.e0, hi = t.e0 + t.n;
-    const int64_t a0 = t.e0 & ~int64_t(kVec - 1);
+    const int64_t a0 = t.e0 & ~int64_t(kAlign - 1);
 
     // Pass 1: full update, weights written, absmax accumulated.
-    uint32_t am = 0u, ar = 0u;
-    for (int64_t vb = a0 + (int64_t)kVec * tid; vb < hi; vb += kTile) {
-        const int64_t elo = max(vb, lo), ehi = min(vb + kVec, hi);
-        const bool full = (elo == vb) && (ehi == vb + kVec);
-        Vec16 x;
-        load_vec(x, vb, lo, hi, full, true, master, grad, mq, vq);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            float m, r;
-            new_m_r(gval(x.g, i), (float)(int8_t)byte_of(x.mq, i), (float)byte_of(x.vq, i), dqm, dqv, c, m, r);
-            x.p[i] = new_p(x.p[i], m, r, c);
-            const int64_t e = vb + i;
-            if (full || (e >= lo && e < hi)) {
-                am = max(am, __float_as_uint(fabsf(m)));
-                ar = max(ar, __float_as_uint(r));
-            }
-        }
-        store_p_bf16(x.p, vb, lo, hi, full, master, param);
+    float am = 0.f, ar = 0.f;
+    for (int64_t vb = a0 + (int64_t)kV * tid; vb < hi; vb += kTile) {
+        if (vb >= lo && vb + kV <= hi)
+            large_pass1_vec<true>(vb, lo, hi, dqm, dqv, master, param, grad, mq, vq, c, am, ar);
+        else
+            large_pass1_vec<false>(vb, lo, hi, dqm, dqv, master, param, grad, mq, vq, c, am, ar);
     }
-#pragma unroll
-    for (int d = 16; d > 0; d >>= 1) {
-        am = max(am, __shfl_xor_sync(0xffffffffu, am, d));
-        ar = max(ar, __shfl_xor_sync(0xffffffffu, ar, d));
-    }
+    warp_max2(am, ar);
     if (lane == 0) {
         s_red[0][warp] = am;
         s_red[1][warp] = ar;
     }
     __syncthreads();
     if (tid == 0) {
-        uint32_t a = 0u, bb = 0u;
+        float a = 0.f, b = 0.f;
         for (int w = 0; w < kThreads / 32; ++w) {
-            a = max(a, s_red[0][w]);
-            bb = max(bb, s_red[1][w]);
+            a = fmaxf(a, s_red[0][w]);
+            b = fmaxf(b, s_red[1][w]);
         }
-        const float AMm = __uint_as_float(a), AMr = __uint_as_float(bb);
-        s_q[0] = AMm > 0.f ? __fdiv_rn(127.f, AMm) : 0.f;
-        s_q[1] = AMr > 0.f ? __fdiv_rn(255.f, AMr) : 0.f;
-        scales[t.blk0] = make_float2(AMm, AMr);
+        s_q[0] = a > 0.f ? __fdiv_rn(127.f, a) : 0.f;
+        s_q[1] = b > 0.f ? __fdiv_rn(255.f, b) : 0.f;
+        scales[t.blk0] = make_float2(a, b);
     }
     __syncthreads();
     const float qm = s_q[0], qv = s_q[1];
 
     // Pass 2: recompute m and sqrt(v) from the unchanged grad and old codes.
-    for (int64_t vb = a0 + (int64_t)kVec * tid; vb < hi; vb += kTile) {
-        const int64_t elo = max(vb, lo), ehi = min(vb + kVec, hi);
-        const bool full = (elo == vb) && (ehi == vb + kVec);
-        Vec16 x;
-        load_vec(x, vb, lo, hi, full, false, master, grad, mq, vq);
-        uint32_t cm[4] = {0, 0, 0, 0}, cv[4] = {0, 0, 0, 0};
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            float m, r;
-            new_m_r(gval(x.g, i), (float)(int8_t)byte_of(x.mq, i), (float)byte_of(x.vq, i), dqm, dqv, c, m, r);
-            cm[i >> 2] |= code_m(m, qm) << (8 * (i & 3));
-            cv[i >> 2] |= code_v(r, qv) << (8 * (i & 3));
-        }
-        store_codes(cm, cv, vb, lo, hi, full, mq, vq);
+    for (int64_t vb = a0 + (int64_t)kV * tid; vb < hi; vb += kTile) {
+        if (vb >= lo && vb + kV <= hi)
+            large_pass2_vec<true>(vb, lo, hi, dqm, dqv, qm, qv, grad, mq, vq, c);
+        else
+            large_pass2_vec<false>(vb, lo, hi, dqm, dqv, qm, qv, grad, mq, vq, c);
     }
 }
 
 __device__ void zero_tile(const Tile& t, uint16_t* param) {
     const int64_t lo = t.e0, hi = t.e0 + t.n;
-    const int64_t a0 = t.e0 & ~int64_t(kVec - 1);
-    for (int64_t vb = a0 + (int64_t)kVec * threadIdx.x; vb < hi; vb += kTile) {
-        if (vb >= lo && vb + kVec <= hi) {
-            uint4* q = reinterpret_cast<uint4*>(param + vb);
-            __stcs(q, make_uint4(0, 0, 0, 0));
-            __stcs(q + 1, make_uint4(0, 0, 0, 0));
+    const int64_t a0 = t.e0 & ~int64_t(kAlign - 1);
+    for (int64_t vb = a0 + (int64_t)kV * threadIdx.x; vb < hi; vb += kTile) {
+        if (vb >= lo && vb + kV <= hi) {
+            __stcs(reinterpret_cast<uint4*>(param + vb), make_uint4(0, 0, 0, 0));
         } else {
-            for (int i = 0; i < kVec; ++i)
+            for (int i = 0; i < kV; ++i)
                 if (vb + i >= lo && vb + i < hi) param[vb + i] = 0;
         }
     }
 }
 
-__global__ void __launch_bounds__(kThreads) adam8_step_kernel(const Tile* __restrict__ tiles, int64_t n_tiles,
+__global__ void __launch_bounds__(kThreads, 2) adam8_step_kernel(const Tile* __restrict__ tiles, int64_t n_tiles,
                                                               int64_t bucket, float* master, uint16_t* param,
                                                               const uint16_t* __restrict__ grad, int8_t* mq,
                                                               uint8_t* vq, float2* scales, int64_t n_blocks,
@@ -546,7 +590,7 @@ __global__ void __launch_bounds__(kThreads) adam8_step_kernel(const Tile* __rest
     // never accessed.
     if (t.e0 < 0 || t.n < 0 || t.e0 + t.n > bucket ||
         (t.kind != TILE_ZERO && (t.blk0 < 0 || t.blk0 + t.nblk > n_blocks)) ||
-        (t.kind == TILE_WHOLE && (t.b <= 0 || t.nblk > kMaxBlk || (t.e0 & (kVec - 1)) + t.n > kTile))) {
+        (t.kind == TILE_WHOLE && (t.b <= 0 || t.nblk > kMaxBlk || (t.e0 & (kAlign - 1)) + t.n > kTile))) {
         if (threadIdx.x == 0) set_status(status, 2);
         return;
     }
@@ -667,17 +711,17 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(PackPtrs ptrs, const
 }
 
 StepC make_step_constants(const dbuf_adam_hparams& hp, float grad_scale) {
-    const double B1 = hp.beta1, B2 = hp.beta2, lr = hp.lr, wd = hp.weight_decay, t = (double)hp.step;
+    const double B1 = hp.beta1, B2 = hp.beta2, lr = hp.lr, wd = hp.weight_decay, eps = hp.eps;
+    const double t = (double)hp.step;
     const double bc1 = 1.0 - std::pow(B1, t);
-    const double bc2 = 1.0 - std::pow(B2, t);
+    const double sq2 = std::sqrt(1.0 - std::pow(B2, t));
     StepC c;
     c.b1 = (float)B1;
     c.omb1 = (float)(1.0 - B1);
     c.b2 = (float)B2;
     c.omb2 = (float)(1.0 - B2);
-    c.bc2s = (float)std::sqrt(bc2);
-    c.eps = hp.eps;
-    c.step = (float)(lr / bc1);
+    c.eps_hat = (float)(eps * sq2);
+    c.step_hat = (float)(lr * sq2 / bc1);
     c.decay = (float)(1.0 - lr * wd);
     c.gscale = grad_scale;
     return c;
@@ -724,7 +768,7 @@ extern "C" dbuf_status dbuf_create(const dbuf_plan_t* plan, void* device_base, s
     if (!out) return fail(DBUF_EINVAL, "dbuf_create: out is NULL");
     *out = nullptr;
     if (!plan) return fail(DBUF_EINVAL, "dbuf_create: plan is NULL");
-    if (plan->align % kVec != 0)
+    if (plan->align % kAlign != 0)
         return fail(DBUF_EINVAL, "dbuf_create: plan alignment must be a multiple of 16 elements");
     dbuf_s* db = new (std::nothrow) dbuf_s;
     if (!db) return fail(DBUF_ENOMEM, "dbuf_create: out of host memory");
