@@ -388,37 +388,62 @@ __device__ __forceinline__ void warp_max2(float& a, float& b) {
     }
 }
 
-// Non-negative floats order like their bit patterns, so the block maxima
-// are kept as unsigned integers for atomicMax in shared memory.
+// Phase 1 of a whole-block tile for one thread-vector: load, update, write
+// the weights.  No barrier in here: FULL and partial vectors of one warp run
+// different instances of this function.
 template <bool FULL>
-__device__ __forceinline__ void whole_vec(const Tile& t, int64_t vb, int64_t lo, int64_t hi, bool multi,
-                                          float* master, uint16_t* param, const uint16_t* grad, int8_t* mq,
-                                          uint8_t* vq, const StepC& c, const float* s_dqm, const float* s_dqv,
-                                          const float* s_qm, const float* s_qv, uint32_t* s_am, uint32_t* s_ar) {
+__device__ __forceinline__ void whole_phase1(int64_t vb, int64_t lo, int64_t hi, int bf, bool one, uint32_t b,
+                                             float* master, uint16_t* param, const uint16_t* grad,
+                                             const int8_t* mq, const uint8_t* vq, const StepC& c,
+                                             const float* s_dqm, const float* s_dqv, int* blk, float* m, float* r) {
+    float dqm[kV], dqv[kV];
+    In8 x;
+    load8<FULL>(x, vb, lo, hi, true, master, grad, mq, vq);
+#pragma unroll
+    for (int i = 0; i < kV; ++i) {
+        const int64_t e = vb + i;
+        blk[i] = (one || e < lo || e >= hi) ? bf : (int)((uint32_t)(e - lo) / b);
+        dqm[i] = s_dqm[blk[i]];
+        dqv[i] = s_dqv[blk[i]];
+    }
+    update8(x, dqm, dqv, c, m, r);
+    store_p8<FULL>(x.p, vb, lo, hi, master, param);
+}
+
+// Up to 256 whole blocks of one tensor.  Non-negative floats order like
+// their bit patterns, so block maxima are kept as unsigned integers for
+// atomicMax in shared memory.
+__device__ void whole_tile(const Tile& t, float* master, uint16_t* param, const uint16_t* grad, int8_t* mq,
+                           uint8_t* vq, float2* scales, const StepC& c) {
+    __shared__ float s_dqm[kMaxBlk], s_dqv[kMaxBlk], s_qm[kMaxBlk], s_qv[kMaxBlk];
+    __shared__ uint32_t s_am[kMaxBlk], s_ar[kMaxBlk];
     const int tid = threadIdx.x;
+    if (tid < t.nblk) {
+        const float2 sc = scales[t.blk0 + tid];
+        s_dqm[tid] = __fdiv_rn(sc.x, 127.f);
+        s_dqv[tid] = __fdiv_rn(sc.y, 255.f);
+        s_am[tid] = 0u;
+        s_ar[tid] = 0u;
+    }
+    __syncthreads();
+    const int64_t lo = t.e0, hi = t.e0 + t.n;
+    const int64_t vb = (t.e0 & ~int64_t(kAlign - 1)) + (int64_t)kV * tid;
     const int64_t elo = max(vb, lo), ehi = min(vb + kV, hi);
     const bool any = elo < ehi;
+    const bool full = (vb >= lo) && (vb + kV <= hi);
     const uint32_t b = (uint32_t)t.b;
-    // block of each element (all equal unless blocks are shorter than a vector
-    // or start off the 8-element grid)
+    const bool multi = t.nblk > 1;
+    // block of the first and last element (all equal unless blocks are
+    // shorter than a vector or start off the 8-element grid)
     const int bf = any ? (multi ? (int)((uint32_t)(elo - lo) / b) : 0) : -1;
     const int bl = any ? (multi ? (int)((uint32_t)(ehi - 1 - lo) / b) : 0) : -1;
     const bool one = (bf == bl);
     int blk[kV];
-    float dqm[kV], dqv[kV], m[kV], r[kV];
-    In8 x;
-    if (any) {
-        load8<FULL>(x, vb, lo, hi, true, master, grad, mq, vq);
-#pragma unroll
-        for (int i = 0; i < kV; ++i) {
-            const int64_t e = vb + i;
-            blk[i] = (one || e < lo || e >= hi) ? bf : (int)((uint32_t)(e - lo) / b);
-            dqm[i] = s_dqm[blk[i]];
-            dqv[i] = s_dqv[blk[i]];
-        }
-        update8(x, dqm, dqv, c, m, r);
-        store_p8<FULL>(x.p, vb, lo, hi, master, param);
-    }
+    float m[kV], r[kV];
+    if (full)
+        whole_phase1<true>(vb, lo, hi, bf, one, b, master, param, grad, mq, vq, c, s_dqm, s_dqv, blk, m, r);
+    else if (any)
+        whole_phase1<false>(vb, lo, hi, bf, one, b, master, param, grad, mq, vq, c, s_dqm, s_dqv, blk, m, r);
     // absmax per block (elements outside the tile have m = r = 0)
     float am = 0.f, ar = 0.f;
     if (any && one) {
@@ -442,8 +467,9 @@ __device__ __forceinline__ void whole_vec(const Tile& t, int64_t vb, int64_t lo,
     __syncthreads();
     if (tid < t.nblk) {
         const float AMm = __uint_as_float(s_am[tid]), AMr = __uint_as_float(s_ar[tid]);
-        const_cast<float*>(s_qm)[tid] = AMm > 0.f ? __fdiv_rn(127.f, AMm) : 0.f;
-        const_cast<float*>(s_qv)[tid] = AMr > 0.f ? __fdiv_rn(255.f, AMr) : 0.f;
+        s_qm[tid] = AMm > 0.f ? __fdiv_rn(127.f, AMm) : 0.f;
+        s_qv[tid] = AMr > 0.f ? __fdiv_rn(255.f, AMr) : 0.f;
+        scales[t.blk0 + tid] = make_float2(AMm, AMr);
     }
     __syncthreads();
     if (any) {
@@ -453,32 +479,11 @@ __device__ __forceinline__ void whole_vec(const Tile& t, int64_t vb, int64_t lo,
             qm[i] = s_qm[blk[i]];
             qv[i] = s_qv[blk[i]];
         }
-        store_codes8<FULL>(m, r, qm, qv, vb, lo, hi, mq, vq);
+        if (full)
+            store_codes8<true>(m, r, qm, qv, vb, lo, hi, mq, vq);
+        else
+            store_codes8<false>(m, r, qm, qv, vb, lo, hi, mq, vq);
     }
-}
-
-__device__ void whole_tile(const Tile& t, float* master, uint16_t* param, const uint16_t* grad, int8_t* mq,
-                           uint8_t* vq, float2* scales, const StepC& c) {
-    __shared__ float s_dqm[kMaxBlk], s_dqv[kMaxBlk], s_qm[kMaxBlk], s_qv[kMaxBlk];
-    __shared__ uint32_t s_am[kMaxBlk], s_ar[kMaxBlk];
-    const int tid = threadIdx.x;
-    if (tid < t.nblk) {
-        const float2 sc = scales[t.blk0 + tid];
-        s_dqm[tid] = __fdiv_rn(sc.x, 127.f);
-        s_dqv[tid] = __fdiv_rn(sc.y, 255.f);
-        s_am[tid] = 0u;
-        s_ar[tid] = 0u;
-    }
-    __syncthreads();
-    const int64_t lo = t.e0, hi = t.e0 + t.n;
-    const int64_t vb = (t.e0 & ~int64_t(kAlign - 1)) + (int64_t)kV * tid;
-    const bool full = (vb >= lo) && (vb + kV <= hi);
-    const bool multi = t.nblk > 1;
-    if (full)
-        whole_vec<true>(t, vb, lo, hi, multi, master, param, grad, mq, vq, c, s_dqm, s_dqv, s_qm, s_qv, s_am, s_ar);
-    else
-        whole_vec<false>(t, vb, lo, hi, multi, master, param, grad, mq, vq, c, s_dqm, s_dqv, s_qm, s_qv, s_am, s_ar);
-    if (tid < t.nblk) scales[t.blk0 + tid] = make_float2(__uint_as_float(s_am[tid]), __uint_as_float(s_ar[tid]));
 }
 
 template <bool FULL>
