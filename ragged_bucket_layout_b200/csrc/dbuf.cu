@@ -388,26 +388,70 @@ __device__ __forceinline__ void warp_max2(float& a, float& b) {
     }
 }
 
-// Phase 1 of a whole-block tile for one thread-vector: load, update, write
-// the weights.  No barrier in here: FULL and partial vectors of one warp run
-// different instances of this function.
+// Phase 1 of a whole-block tile for a thread-vector that lies in one block:
+// load, update, write the weights.  No barrier in here: FULL and partial
+// vectors of one warp run different instances of this function.
 template <bool FULL>
-__device__ __forceinline__ void whole_phase1(int64_t vb, int64_t lo, int64_t hi, int bf, bool one, uint32_t b,
-                                             float* master, uint16_t* param, const uint16_t* grad,
-                                             const int8_t* mq, const uint8_t* vq, const StepC& c,
-                                             const float* s_dqm, const float* s_dqv, int* blk, float* m, float* r) {
-    float dqm[kV], dqv[kV];
+__device__ __forceinline__ void phase1_one(int64_t vb, int64_t lo, int64_t hi, float dqm, float dqv, float* master,
+                                           uint16_t* param, const uint16_t* grad, const int8_t* mq,
+                                           const uint8_t* vq, const StepC& c, float* m, float* r) {
     In8 x;
     load8<FULL>(x, vb, lo, hi, true, master, grad, mq, vq);
 #pragma unroll
     for (int i = 0; i < kV; ++i) {
-        const int64_t e = vb + i;
-        blk[i] = (one || e < lo || e >= hi) ? bf : (int)((uint32_t)(e - lo) / b);
-        dqm[i] = s_dqm[blk[i]];
-        dqv[i] = s_dqv[blk[i]];
+        new_m_r(g_of(x, i), sbyte_to_f(x.mq[i >> 2], i & 3), ubyte_to_f(x.vq[i >> 2], i & 3), dqm, dqv, c, m[i],
+                r[i]);
+        x.p[i] = new_p(x.p[i], m[i], r[i], c);
     }
-    update8(x, dqm, dqv, c, m, r);
     store_p8<FULL>(x.p, vb, lo, hi, master, param);
+}
+
+// The same for a vector that spans several blocks (blocks shorter than 8
+// elements, or off the 8-element grid): per-element block numbers.
+__device__ __noinline__ void phase1_mixed(int64_t vb, int64_t lo, int64_t hi, uint32_t b, int bf, float* master,
+                                          uint16_t* param, const uint16_t* grad, const int8_t* mq,
+                                          const uint8_t* vq, const StepC& c, const float* s_dqm,
+                                          const float* s_dqv, uint32_t* s_am, uint32_t* s_ar, float* m,
+                                          float* r) {
+    In8 x;
+    load8<false>(x, vb, lo, hi, true, master, grad, mq, vq);
+#pragma unroll
+    for (int i = 0; i < kV; ++i) {
+        const int64_t e = vb + i;
+        const int blk = (e < lo || e >= hi) ? bf : (int)((uint32_t)(e - lo) / b);
+        new_m_r(g_of(x, i), sbyte_to_f(x.mq[i >> 2], i & 3), ubyte_to_f(x.vq[i >> 2], i & 3), s_dqm[blk],
+                s_dqv[blk], c, m[i], r[i]);
+        x.p[i] = new_p(x.p[i], m[i], r[i], c);
+        atomicMax(&s_am[blk], __float_as_uint(fabsf(m[i])));
+        atomicMax(&s_ar[blk], __float_as_uint(r[i]));
+    }
+    store_p8<false>(x.p, vb, lo, hi, master, param);
+}
+
+__device__ __noinline__ void codes_mixed(int64_t vb, int64_t lo, int64_t hi, uint32_t b, int bf, const float* s_qm,
+                                         const float* s_qv, const float* m, const float* r, int8_t* mq,
+                                         uint8_t* vq) {
+    float qm[kV], qv[kV];
+#pragma unroll
+    for (int i = 0; i < kV; ++i) {
+        const int64_t e = vb + i;
+        const int blk = (e < lo || e >= hi) ? bf : (int)((uint32_t)(e - lo) / b);
+        qm[i] = s_qm[blk];
+        qv[i] = s_qv[blk];
+    }
+    store_codes8<false>(m, r, qm, qv, vb, lo, hi, mq, vq);
+}
+
+template <bool FULL>
+__device__ __forceinline__ void codes_one(int64_t vb, int64_t lo, int64_t hi, float qm1, float qv1, const float* m,
+                                          const float* r, int8_t* mq, uint8_t* vq) {
+    float qm[kV], qv[kV];
+#pragma unroll
+    for (int i = 0; i < kV; ++i) {
+        qm[i] = qm1;
+        qv[i] = qv1;
+    }
+    store_codes8<FULL>(m, r, qm, qv, vb, lo, hi, mq, vq);
 }
 
 // Up to 256 whole blocks of one tensor.  Non-negative floats order like
@@ -432,37 +476,40 @@ __device__ void whole_tile(const Tile& t, float* master, uint16_t* param, const 
     const bool any = elo < ehi;
     const bool full = (vb >= lo) && (vb + kV <= hi);
     const uint32_t b = (uint32_t)t.b;
-    const bool multi = t.nblk > 1;
-    // block of the first and last element (all equal unless blocks are
-    // shorter than a vector or start off the 8-element grid)
-    const int bf = any ? (multi ? (int)((uint32_t)(elo - lo) / b) : 0) : -1;
-    const int bl = any ? (multi ? (int)((uint32_t)(ehi - 1 - lo) / b) : 0) : -1;
+    const bool single = t.nblk == 1;
+    // block of the first and last element of this vector
+    const int bf = any ? (single ? 0 : (int)((uint32_t)(elo - lo) / b)) : -1;
+    const int bl = any ? (single ? 0 : (int)((uint32_t)(ehi - 1 - lo) / b)) : -1;
     const bool one = (bf == bl);
-    int blk[kV];
-    float m[kV], r[kV];
-    if (full)
-        whole_phase1<true>(vb, lo, hi, bf, one, b, master, param, grad, mq, vq, c, s_dqm, s_dqv, blk, m, r);
-    else if (any)
-        whole_phase1<false>(vb, lo, hi, bf, one, b, master, param, grad, mq, vq, c, s_dqm, s_dqv, blk, m, r);
-    // absmax per block (elements outside the tile have m = r = 0)
-    float am = 0.f, ar = 0.f;
+    float m[kV], r[kV];        // registers (fast path)
+    float mx[kV], rx[kV];      // the mixed path's copies (passed by address)
+    float am = 0.f, ar = 0.f;  // elements outside the tile have m = r = 0
     if (any && one) {
+        const float dqm = s_dqm[bf], dqv = s_dqv[bf];
+        if (full)
+            phase1_one<true>(vb, lo, hi, dqm, dqv, master, param, grad, mq, vq, c, m, r);
+        else
+            phase1_one<false>(vb, lo, hi, dqm, dqv, master, param, grad, mq, vq, c, m, r);
 #pragma unroll
         for (int i = 0; i < kV; ++i) {
             am = fmaxf(am, fabsf(m[i]));
             ar = fmaxf(ar, r[i]);
         }
     } else if (any) {
-#pragma unroll
-        for (int i = 0; i < kV; ++i) {
-            atomicMax(&s_am[blk[i]], __float_as_uint(fabsf(m[i])));
-            atomicMax(&s_ar[blk[i]], __float_as_uint(r[i]));
-        }
+        phase1_mixed(vb, lo, hi, b, bf, master, param, grad, mq, vq, c, s_dqm, s_dqv, s_am, s_ar, mx, rx);
     }
-    const int key = (any && one) ? bf : -1;
-    if (segmented_max(key, am, ar) && key >= 0) {
-        atomicMax(&s_am[key], __float_as_uint(am));
-        atomicMax(&s_ar[key], __float_as_uint(ar));
+    if (single) {
+        warp_max2(am, ar);
+        if ((tid & 31) == 0) {
+            atomicMax(&s_am[0], __float_as_uint(am));
+            atomicMax(&s_ar[0], __float_as_uint(ar));
+        }
+    } else {
+        const int key = (any && one) ? bf : -1;
+        if (segmented_max(key, am, ar) && key >= 0) {
+            atomicMax(&s_am[key], __float_as_uint(am));
+            atomicMax(&s_ar[key], __float_as_uint(ar));
+        }
     }
     __syncthreads();
     if (tid < t.nblk) {
@@ -472,17 +519,14 @@ __device__ void whole_tile(const Tile& t, float* master, uint16_t* param, const 
         scales[t.blk0 + tid] = make_float2(AMm, AMr);
     }
     __syncthreads();
-    if (any) {
-        float qm[kV], qv[kV];
-#pragma unroll
-        for (int i = 0; i < kV; ++i) {
-            qm[i] = s_qm[blk[i]];
-            qv[i] = s_qv[blk[i]];
-        }
+    if (any && one) {
+        const float qm = s_qm[bf], qv = s_qv[bf];
         if (full)
-            store_codes8<true>(m, r, qm, qv, vb, lo, hi, mq, vq);
+            codes_one<true>(vb, lo, hi, qm, qv, m, r, mq, vq);
         else
-            store_codes8<false>(m, r, qm, qv, vb, lo, hi, mq, vq);
+            codes_one<false>(vb, lo, hi, qm, qv, m, r, mq, vq);
+    } else if (any) {
+        codes_mixed(vb, lo, hi, b, bf, s_qm, s_qv, mx, rx, mq, vq);
     }
 }
 
