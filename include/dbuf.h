@@ -174,7 +174,7 @@ dbuf_status dbuf_scales(const dbuf_t* db, float** scales, int64_t* n_blocks);
 dbuf_status dbuf_get_device_status(dbuf_t* db, int32_t* code, void* stream);
 
 /* One entry of the step kernel's work table (introspection for tests and
- * tools; the kernel's own table holds the same entries).  kind 0: up to 256
+ * tools; the kernel's own table holds the same entries).  kind 0: up to 254
  * whole blocks of one tensor, at most 4096 elements counted from the
  * 16-element boundary at or below first_elem; kind 1: one block longer than
  * that, streamed twice; kind 2: a padding range whose bf16 copy is zeroed. */

@@ -1,24 +1,12 @@
-// Device runtime of the ragged-bucket optimizer step (sm_100a).
+// Device runtime of the ragged-bucket optimizer step (sm_100a): the C-ABI
+// of include/dbuf.h apart from the planner (planner.cpp).
 //
 // DBuffer (veScale-FSDP paper Sec. 5, page section "3. DBuffer"): one batch
 // allocation holds every bucket array of a plan; tensors are zero-copy views;
-// group operations run as one launch over the whole bucket.  The fused step
-// is the block-wise 8-bit Adam of the paper's 8-bit Adam case study
-// (Sec. 6.3): each quantisation block (k whole rows) is updated and
-// requantised on its own, which the RaggedShard layout makes possible
-// because no block crosses a slice boundary.
-//
-// Work decomposition (host-built table, uploaded once by dbuf_create):
-//   WHOLE  up to 4096 elements holding up to 256 whole blocks of one tensor;
-//          one CTA keeps the new m and sqrt(v) in registers, reduces each
-//          block's absmax in shared memory, then writes the codes.
-//   LARGE  one block longer than a tile; one CTA streams it twice: pass 1
-//          updates weights and finds the absmax, pass 2 re-reads grad and
-//          codes (an L2 hit while the block is recent), recomputes m and
-//          sqrt(v) bit-identically and writes the codes.
-//   ZERO   a padding range; the bf16 parameter copy is set to zero.
-// Every thread owns 16 consecutive elements (16-element aligned in the
-// bucket), so grad, master, codes and the bf16 copy move as 128-bit accesses.
+// group operations run as one launch over the whole bucket.  The kernels are
+// in step_kernel.cuh (the fused 8-bit Adam step) and pack_kernel.cuh (the
+// copy-in baseline); this file builds their work tables once per bucket and
+// launches them on the caller's stream.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -31,6 +19,9 @@
 #include <vector>
 
 #include "internal.h"
+#include "pack_kernel.cuh"
+#include "step_kernel.cuh"
+#include "tables.h"
 
 // ------------------------------------------------------------------ errors
 
@@ -58,38 +49,7 @@ extern "C" const char* dbuf_last_error(void) { return dbuf_detail::g_err.c_str()
 
 namespace {
 
-constexpr int kThreads = 512;          // threads per CTA of the step kernel
-constexpr int kAlign = 16;             // tensor starts are multiples of 16 elements
-constexpr int kTile = 4096;            // elements per tile (8 per thread)
-constexpr int kMaxBlk = 256;           // blocks per WHOLE tile
-constexpr int64_t kZeroChunk = 65536;  // elements per ZERO tile
-constexpr int64_t kPackChunk = 16384;  // elements per copy-in CTA (32 KB)
-constexpr int kPackThreads = 256;
-constexpr int kMaxPackPtrs = 1024;     // tensor pointers passed by value per launch
-
-enum : int32_t { TILE_WHOLE = 0, TILE_LARGE = 1, TILE_ZERO = 2 };
-
-struct Tile {
-    int64_t e0;    // first bucket element of the tile
-    int64_t blk0;  // index of its first block (scale index)
-    int64_t n;     // elements in the tile
-    int32_t b;     // block size (WHOLE), 0 otherwise
-    int32_t kind;
-    int32_t nblk;  // blocks in the tile (WHOLE)
-    int32_t pad_;
-};
-static_assert(sizeof(Tile) == 40, "tile layout");
-
-struct PackChunk {
-    int64_t src_off;  // element offset in the source tensor
-    int64_t dst_off;  // element offset in the bucket
-    int32_t tensor;   // caller's tensor index
-    int32_t count;    // elements
-};
-
-struct PackPtrs {
-    const uint16_t* p[kMaxPackPtrs];
-};
+using namespace dbuf_k;
 
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -189,575 +149,14 @@ struct dbuf_s {
     std::vector<Tile> h_tiles;
     std::vector<PackChunk> h_chunks;
     std::vector<int64_t> h_chunk_first;
+    int step_grid = 0;  // persistent CTAs of the step kernel
 };
 
-// ----------------------------------------------------------- device code
+// ----------------------------------------------------------- launches
 
 namespace {
 
-// Per-step scalars (formed on the host in double, rounded to float once).
-// The bias corrections are folded into the step size and eps:
-//   (lr/bc1) m / (sqrt(v)/sqrt(bc2) + eps) = step_hat * m / (sqrt(v) + eps_hat).
-struct StepC {
-    float b1, omb1, b2, omb2, eps_hat, step_hat, decay, gscale;
-};
-
-constexpr int kV = 8;  // elements per thread-vector in the step kernel
-
-__device__ __forceinline__ void set_status(int32_t* status, int32_t code) { atomicCAS(status, 0, code); }
-
-__device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) { return __uint_as_float(h << 16); }
-
-// Code bytes to float without the conversion unit: a byte b placed in the
-// low mantissa bits of 2^23 reads as 2^23 + b; subtracting 2^23 is exact.
-// int8 codes are stored with the sign bit flipped first (b = code + 128).
-__device__ __forceinline__ float ubyte_to_f(uint32_t w, uint32_t sel) {
-    return __fsub_rn(__uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540u | sel)), 8388608.0f);
-}
-__device__ __forceinline__ float sbyte_to_f(uint32_t w_flipped, uint32_t sel) {
-    return __fsub_rn(__uint_as_float(__byte_perm(w_flipped, 0x4B000000u, 0x7540u | sel)), 8388736.0f);
-}
-
-// Round to the nearest integer, ties to even, by adding 1.5*2^23: the sum
-// lies where the float spacing is 1, so the addition itself rounds; the
-// low byte of the result's bits is the integer's two's-complement low byte.
-// Valid for |x| < 2^22; the codes here satisfy |x| <= 255.
-__device__ __forceinline__ uint32_t rne_low_bits(float x) { return __float_as_uint(__fadd_rn(x, 12582912.0f)); }
-
-__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-    return __byte_perm(__byte_perm(a, b, 0x0040u), __byte_perm(c, d, 0x0040u), 0x5410u);
-}
-
-__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&h);
-}
-
-// New m and sqrt(v) of one element, every operation rounded on its own.
-__device__ __forceinline__ void new_m_r(float graw, float qmf, float qvf, float dqm, float dqv, const StepC& c,
-                                        float& m, float& r) {
-    const float g = __fmul_rn(graw, c.gscale);
-    const float mo = __fmul_rn(qmf, dqm);
-    const float so = __fmul_rn(qvf, dqv);
-    const float vo = __fmul_rn(so, so);
-    m = __fadd_rn(__fmul_rn(c.b1, mo), __fmul_rn(c.omb1, g));
-    const float v = __fadd_rn(__fmul_rn(c.b2, vo), __fmul_rn(c.omb2, __fmul_rn(g, g)));
-    r = __fsqrt_rn(v);
-}
-
-__device__ __forceinline__ float new_p(float p, float m, float r, const StepC& c) {
-    const float u = __fdiv_rn(m, __fadd_rn(r, c.eps_hat));
-    return __fsub_rn(__fmul_rn(p, c.decay), __fmul_rn(c.step_hat, u));
-}
-
-// Inputs of one thread-vector (8 consecutive bucket elements).
-struct In8 {
-    uint32_t g[4];   // bf16 pairs
-    float p[8];
-    uint32_t mq[2];  // int8 codes with the sign bit flipped
-    uint32_t vq[2];  // uint8 codes
-};
-
-// Load elements [vb, vb+8); when !FULL only those in [lo, hi) are read and
-// the rest are zero.
-template <bool FULL>
-__device__ __forceinline__ void load8(In8& x, int64_t vb, int64_t lo, int64_t hi, bool want_p, const float* master,
-                                      const uint16_t* grad, const int8_t* mq, const uint8_t* vq) {
-    if (FULL) {
-        const uint4 g = __ldg(reinterpret_cast<const uint4*>(grad + vb));
-        x.g[0] = g.x; x.g[1] = g.y; x.g[2] = g.z; x.g[3] = g.w;
-        const uint2 a = *reinterpret_cast<const uint2*>(mq + vb);
-        const uint2 b = *reinterpret_cast<const uint2*>(vq + vb);
-        x.mq[0] = a.x ^ 0x80808080u; x.mq[1] = a.y ^ 0x80808080u;
-        x.vq[0] = b.x; x.vq[1] = b.y;
-        if (want_p) {
-            const float4 p0 = __ldcs(reinterpret_cast<const float4*>(master + vb));
-            const float4 p1 = __ldcs(reinterpret_cast<const float4*>(master + vb) + 1);
-            x.p[0] = p0.x; x.p[1] = p0.y; x.p[2] = p0.z; x.p[3] = p0.w;
-            x.p[4] = p1.x; x.p[5] = p1.y; x.p[6] = p1.z; x.p[7] = p1.w;
-        }
-    } else {
-        uint32_t g[4] = {0, 0, 0, 0}, a[2] = {0, 0}, b[2] = {0, 0};
-#pragma unroll
-        for (int i = 0; i < kV; ++i) {
-            const int64_t e = vb + i;
-            const bool in = (e >= lo && e < hi);
-            x.p[i] = (in && want_p) ? master[e] : 0.f;
-            if (in) {
-                g[i >> 1] |= (uint32_t)grad[e] << (16 * (i & 1));
-                a[i >> 2] |= (uint32_t)(uint8_t)mq[e] << (8 * (i & 3));
-                b[i >> 2] |= (uint32_t)vq[e] << (8 * (i & 3));
-            }
-        }
-        x.g[0] = g[0]; x.g[1] = g[1]; x.g[2] = g[2]; x.g[3] = g[3];
-        x.mq[0] = a[0] ^ 0x80808080u; x.mq[1] = a[1] ^ 0x80808080u;
-        x.vq[0] = b[0]; x.vq[1] = b[1];
-    }
-}
-
-__device__ __forceinline__ float g_of(const In8& x, int i) {
-    const uint32_t w = x.g[i >> 1];
-    return __uint_as_float((i & 1) ? (w & 0xffff0000u) : (w << 16));
-}
-
-// Update 8 elements; dq* are per element (equal when the vector lies in one block).
-__device__ __forceinline__ void update8(In8& x, const float* dqm, const float* dqv, const StepC& c, float* m,
-                                        float* r) {
-#pragma unroll
-    for (int i = 0; i < kV; ++i) {
-        new_m_r(g_of(x, i), sbyte_to_f(x.mq[i >> 2], i & 3), ubyte_to_f(x.vq[i >> 2], i & 3), dqm[i], dqv[i], c, m[i],
-                r[i]);
-        x.p[i] = new_p(x.p[i], m[i], r[i], c);
-    }
-}
-
-template <bool FULL>
-__device__ __forceinline__ void store_p8(const float* p, int64_t vb, int64_t lo, int64_t hi, float* master,
-                                         uint16_t* param) {
-    const uint4 h = make_uint4(bf16x2_bits(p[0], p[1]), bf16x2_bits(p[2], p[3]), bf16x2_bits(p[4], p[5]),
-                               bf16x2_bits(p[6], p[7]));
-    if (FULL) {
-        __stcs(reinterpret_cast<float4*>(master + vb), make_float4(p[0], p[1], p[2], p[3]));
-        __stcs(reinterpret_cast<float4*>(master + vb) + 1, make_float4(p[4], p[5], p[6], p[7]));
-        __stcs(reinterpret_cast<uint4*>(param + vb), h);
-    } else {
-        const uint32_t hw[4] = {h.x, h.y, h.z, h.w};
-#pragma unroll
-        for (int i = 0; i < kV; ++i) {
-            const int64_t e = vb + i;
-            if (e >= lo && e < hi) {
-                master[e] = p[i];
-                param[e] = (uint16_t)(hw[i >> 1] >> (16 * (i & 1)));
-            }
-        }
-    }
-}
-
-// Codes of 8 elements from m, r and the per-element quotients 127/absmax,
-// 255/absmax.  |m*qm| <= 127 and 0 <= r*qv <= 255 hold by construction
-// (absmax over the same values), so rounding never needs a clamp.
-template <bool FULL>
-__device__ __forceinline__ void store_codes8(const float* m, const float* r, const float* qm, const float* qv,
-                                             int64_t vb, int64_t lo, int64_t hi, int8_t* mq, uint8_t* vq) {
-    uint32_t bm[kV], bv[kV];
-#pragma unroll
-    for (int i = 0; i < kV; ++i) {
-        bm[i] = rne_low_bits(__fmul_rn(m[i], qm[i]));
-        bv[i] = rne_low_bits(__fmul_rn(r[i], qv[i]));
-    }
-    const uint2 cm = make_uint2(pack_low_bytes(bm[0], bm[1], bm[2], bm[3]), pack_low_bytes(bm[4], bm[5], bm[6], bm[7]));
-    const uint2 cv = make_uint2(pack_low_bytes(bv[0], bv[1], bv[2], bv[3]), pack_low_bytes(bv[4], bv[5], bv[6], bv[7]));
-    if (FULL) {
-        __stcs(reinterpret_cast<uint2*>(mq + vb), cm);
-        __stcs(reinterpret_cast<uint2*>(vq + vb), cv);
-    } else {
-#pragma unroll
-        for (int i = 0; i < kV; ++i) {
-            const int64_t e = vb + i;
-            if (e >= lo && e < hi) {
-                mq[e] = (int8_t)(bm[i] & 0xffu);
-                vq[e] = (uint8_t)(bv[i] & 0xffu);
-            }
-        }
-    }
-}
-
-// Max over the lanes of a warp that share `key`, where lanes with equal keys
-// are contiguous; the first lane of each run ends with the run's maximum.
-__device__ __forceinline__ bool segmented_max(int key, float& a, float& b) {
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        const int ok = __shfl_down_sync(0xffffffffu, key, d);
-        const float oa = __shfl_down_sync(0xffffffffu, a, d);
-        const float ob = __shfl_down_sync(0xffffffffu, b, d);
-        if (lane + d < 32 && ok == key) {
-            a = fmaxf(a, oa);
-            b = fmaxf(b, ob);
-        }
-    }
-    const int prev = __shfl_up_sync(0xffffffffu, key, 1);
-    return (lane == 0) || (prev != key);
-}
-
-__device__ __forceinline__ void warp_max2(float& a, float& b) {
-#pragma unroll
-    for (int d = 16; d > 0; d >>= 1) {
-        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, d));
-        b = fmaxf(b, __shfl_xor_sync(0xffffffffu, b, d));
-    }
-}
-
-// Phase 1 of a whole-block tile for a thread-vector that lies in one block:
-// load, update, write the weights.  No barrier in here: FULL and partial
-// vectors of one warp run different instances of this function.
-template <bool FULL>
-__device__ __forceinline__ void phase1_one(int64_t vb, int64_t lo, int64_t hi, float dqm, float dqv, float* master,
-                                           uint16_t* param, const uint16_t* grad, const int8_t* mq,
-                                           const uint8_t* vq, const StepC& c, float* m, float* r) {
-    In8 x;
-    load8<FULL>(x, vb, lo, hi, true, master, grad, mq, vq);
-#pragma unroll
-    for (int i = 0; i < kV; ++i) {
-        new_m_r(g_of(x, i), sbyte_to_f(x.mq[i >> 2], i & 3), ubyte_to_f(x.vq[i >> 2], i & 3), dqm, dqv, c, m[i],
-                r[i]);
-        x.p[i] = new_p(x.p[i], m[i], r[i], c);
-    }
-    store_p8<FULL>(x.p, vb, lo, hi, master, param);
-}
-
-// The same for a vector that spans several blocks (blocks shorter than 8
-// elements, or off the 8-element grid): per-element block numbers.
-__device__ __noinline__ void phase1_mixed(int64_t vb, int64_t lo, int64_t hi, uint32_t b, int bf, float* master,
-                                          uint16_t* param, const uint16_t* grad, const int8_t* mq,
-                                          const uint8_t* vq, const StepC& c, const float* s_dqm,
-                                          const float* s_dqv, uint32_t* s_am, uint32_t* s_ar, float* m,
-                                          float* r) {
-    In8 x;
-    load8<false>(x, vb, lo, hi, true, master, grad, mq, vq);
-#pragma unroll
-    for (int i = 0; i < kV; ++i) {
-        const int64_t e = vb + i;
-        const int blk = (e < lo || e >= hi) ? bf : (int)((uint32_t)(e - lo) / b);
-        new_m_r(g_of(x, i), sbyte_to_f(x.mq[i >> 2], i & 3), ubyte_to_f(x.vq[i >> 2], i & 3), s_dqm[blk],
-                s_dqv[blk], c, m[i], r[i]);
-        x.p[i] = new_p(x.p[i], m[i], r[i], c);
-        atomicMax(&s_am[blk], __float_as_uint(fabsf(m[i])));
-        atomicMax(&s_ar[blk], __float_as_uint(r[i]));
-    }
-    store_p8<false>(x.p, vb, lo, hi, master, param);
-}
-
-__device__ __noinline__ void codes_mixed(int64_t vb, int64_t lo, int64_t hi, uint32_t b, int bf, const float* s_qm,
-                                         const float* s_qv, const float* m, const float* r, int8_t* mq,
-                                         uint8_t* vq) {
-    float qm[kV], qv[kV];
-#pragma unroll
-    for (int i = 0; i < kV; ++i) {
-        const int64_t e = vb + i;
-        const int blk = (e < lo || e >= hi) ? bf : (int)((uint32_t)(e - lo) / b);
-        qm[i] = s_qm[blk];
-        qv[i] = s_qv[blk];
-    }
-    store_codes8<false>(m, r, qm, qv, vb, lo, hi, mq, vq);
-}
-
-template <bool FULL>
-__device__ __forceinline__ void codes_one(int64_t vb, int64_t lo, int64_t hi, float qm1, float qv1, const float* m,
-                                          const float* r, int8_t* mq, uint8_t* vq) {
-    float qm[kV], qv[kV];
-#pragma unroll
-    for (int i = 0; i < kV; ++i) {
-        qm[i] = qm1;
-        qv[i] = qv1;
-    }
-    store_codes8<FULL>(m, r, qm, qv, vb, lo, hi, mq, vq);
-}
-
-// Up to 256 whole blocks of one tensor.  Non-negative floats order like
-// their bit patterns, so block maxima are kept as unsigned integers for
-// atomicMax in shared memory.
-__device__ void whole_tile(const Tile& t, float* master, uint16_t* param, const uint16_t* grad, int8_t* mq,
-                           uint8_t* vq, float2* scales, const StepC& c) {
-    __shared__ float s_dqm[kMaxBlk], s_dqv[kMaxBlk], s_qm[kMaxBlk], s_qv[kMaxBlk];
-    __shared__ uint32_t s_am[kMaxBlk], s_ar[kMaxBlk];
-    const int tid = threadIdx.x;
-    if (tid < t.nblk) {
-        const float2 sc = scales[t.blk0 + tid];
-        s_dqm[tid] = __fdiv_rn(sc.x, 127.f);
-        s_dqv[tid] = __fdiv_rn(sc.y, 255.f);
-        s_am[tid] = 0u;
-        s_ar[tid] = 0u;
-    }
-    __syncthreads();
-    const int64_t lo = t.e0, hi = t.e0 + t.n;
-    const int64_t vb = (t.e0 & ~int64_t(kAlign - 1)) + (int64_t)kV * tid;
-    const int64_t elo = max(vb, lo), ehi = min(vb + kV, hi);
-    const bool any = elo < ehi;
-    const bool full = (vb >= lo) && (vb + kV <= hi);
-    const uint32_t b = (uint32_t)t.b;
-    const bool single = t.nblk == 1;
-    // block of the first and last element of this vector
-    const int bf = any ? (single ? 0 : (int)((uint32_t)(elo - lo) / b)) : -1;
-    const int bl = any ? (single ? 0 : (int)((uint32_t)(ehi - 1 - lo) / b)) : -1;
-    const bool one = (bf == bl);
-    float m[kV], r[kV];        // registers (fast path)
-    float mx[kV], rx[kV];      // the mixed path's copies (passed by address)
-    float am = 0.f, ar = 0.f;  // elements outside the tile have m = r = 0
-    if (any && one) {
-        const float dqm = s_dqm[bf], dqv = s_dqv[bf];
-        if (full)
-            phase1_one<true>(vb, lo, hi, dqm, dqv, master, param, grad, mq, vq, c, m, r);
-        else
-            phase1_one<false>(vb, lo, hi, dqm, dqv, master, param, grad, mq, vq, c, m, r);
-#pragma unroll
-        for (int i = 0; i < kV; ++i) {
-            am = fmaxf(am, fabsf(m[i]));
-            ar = fmaxf(ar, r[i]);
-        }
-    } else if (any) {
-        phase1_mixed(vb, lo, hi, b, bf, master, param, grad, mq, vq, c, s_dqm, s_dqv, s_am, s_ar, mx, rx);
-    }
-    if (single) {
-        warp_max2(am, ar);
-        if ((tid & 31) == 0) {
-            atomicMax(&s_am[0], __float_as_uint(am));
-            atomicMax(&s_ar[0], __float_as_uint(ar));
-        }
-    } else {
-        const int key = (any && one) ? bf : -1;
-        if (segmented_max(key, am, ar) && key >= 0) {
-            atomicMax(&s_am[key], __float_as_uint(am));
-            atomicMax(&s_ar[key], __float_as_uint(ar));
-        }
-    }
-    __syncthreads();
-    if (tid < t.nblk) {
-        const float AMm = __uint_as_float(s_am[tid]), AMr = __uint_as_float(s_ar[tid]);
-        s_qm[tid] = AMm > 0.f ? __fdiv_rn(127.f, AMm) : 0.f;
-        s_qv[tid] = AMr > 0.f ? __fdiv_rn(255.f, AMr) : 0.f;
-        scales[t.blk0 + tid] = make_float2(AMm, AMr);
-    }
-    __syncthreads();
-    if (any && one) {
-        const float qm = s_qm[bf], qv = s_qv[bf];
-        if (full)
-            codes_one<true>(vb, lo, hi, qm, qv, m, r, mq, vq);
-        else
-            codes_one<false>(vb, lo, hi, qm, qv, m, r, mq, vq);
-    } else if (any) {
-        codes_mixed(vb, lo, hi, b, bf, s_qm, s_qv, mx, rx, mq, vq);
-    }
-}
-
-template <bool FULL>
-__device__ __forceinline__ void large_pass1_vec(int64_t vb, int64_t lo, int64_t hi, float dqm1, float dqv1,
-                                                float* master, uint16_t* param, const uint16_t* grad,
-                                                const int8_t* mq, const uint8_t* vq, const StepC& c, float& am,
-                                                float& ar) {
-    In8 x;
-    float dqm[kV], dqv[kV], m[kV], r[kV];
-#pragma unroll
-    for (int i = 0; i < kV; ++i) {
-        dqm[i] = dqm1;
-        dqv[i] = dqv1;
-    }
-    load8<FULL>(x, vb, lo, hi, true, master, grad, mq, vq);
-    update8(x, dqm, dqv, c, m, r);
-    store_p8<FULL>(x.p, vb, lo, hi, master, param);
-#pragma unroll
-    for (int i = 0; i < kV; ++i) {
-        am = fmaxf(am, fabsf(m[i]));
-        ar = fmaxf(ar, r[i]);
-    }
-}
-
-template <bool FULL>
-__device__ __forceinline__ void large_pass2_vec(int64_t vb, int64_t lo, int64_t hi, float dqm1, float dqv1,
-                                                float qm1, float qv1, const uint16_t* grad, int8_t* mq, uint8_t* vq,
-                                                const StepC& c) {
-    In8 x;
-    float m[kV], r[kV], qm[kV], qv[kV];
-    load8<FULL>(x, vb, lo, hi, false, nullptr, grad, mq, vq);
-#pragma unroll
-    for (int i = 0; i < kV; ++i) {
-        new_m_r(g_of(x, i), sbyte_to_f(x.mq[i >> 2], i & 3), ubyte_to_f(x.vq[i >> 2], i & 3), dqm1, dqv1, c, m[i],
-                r[i]);
-        qm[i] = qm1;
-        qv[i] = qv1;
-    }
-    store_codes8<FULL>(m, r, qm, qv, vb, lo, hi, mq, vq);
-}
-
-__device__ void large_block(const Tile& t, float* master, uint16_t* param, const uint16_t* grad, int8_t* mq,
-                            uint8_t* vq, float2* scales, const StepC& c) {
-    __shared__ float s_red[2][kThreads / 32];
-    __shared__ float s_q[2];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const float2 sc = scales[t.blk0];
-    const float dqm = __fdiv_rn(sc.x, 127.f), dqv = __fdiv_rn(sc.y, 255.f);
-    const int64_t lo = t.e0, hi = t.e0 + t.n;
-    const int64_t a0 = t.e0 & ~int64_t(kAlign - 1);
-
-    // Pass 1: full update, weights written, absmax accumulated.
-    float am = 0.f, ar = 0.f;
-    for (int64_t vb = a0 + (int64_t)kV * tid; vb < hi; vb += kTile) {
-        if (vb >= lo && vb + kV <= hi)
-            large_pass1_vec<true>(vb, lo, hi, dqm, dqv, master, param, grad, mq, vq, c, am, ar);
-        else
-            large_pass1_vec<false>(vb, lo, hi, dqm, dqv, master, param, grad, mq, vq, c, am, ar);
-    }
-    warp_max2(am, ar);
-    if (lane == 0) {
-        s_red[0][warp] = am;
-        s_red[1][warp] = ar;
-    }
-    __syncthreads();
-    if (tid == 0) {
-        float a = 0.f, b = 0.f;
-        for (int w = 0; w < kThreads / 32; ++w) {
-            a = fmaxf(a, s_red[0][w]);
-            b = fmaxf(b, s_red[1][w]);
-        }
-        s_q[0] = a > 0.f ? __fdiv_rn(127.f, a) : 0.f;
-        s_q[1] = b > 0.f ? __fdiv_rn(255.f, b) : 0.f;
-        scales[t.blk0] = make_float2(a, b);
-    }
-    __syncthreads();
-    const float qm = s_q[0], qv = s_q[1];
-
-    // Pass 2: recompute m and sqrt(v) from the unchanged grad and old codes.
-    for (int64_t vb = a0 + (int64_t)kV * tid; vb < hi; vb += kTile) {
-        if (vb >= lo && vb + kV <= hi)
-            large_pass2_vec<true>(vb, lo, hi, dqm, dqv, qm, qv, grad, mq, vq, c);
-        else
-            large_pass2_vec<false>(vb, lo, hi, dqm, dqv, qm, qv, grad, mq, vq, c);
-    }
-}
-
-__device__ void zero_tile(const Tile& t, uint16_t* param) {
-    const int64_t lo = t.e0, hi = t.e0 + t.n;
-    const int64_t a0 = t.e0 & ~int64_t(kAlign - 1);
-    for (int64_t vb = a0 + (int64_t)kV * threadIdx.x; vb < hi; vb += kTile) {
-        if (vb >= lo && vb + kV <= hi) {
-            __stcs(reinterpret_cast<uint4*>(param + vb), make_uint4(0, 0, 0, 0));
-        } else {
-            for (int i = 0; i < kV; ++i)
-                if (vb + i >= lo && vb + i < hi) param[vb + i] = 0;
-        }
-    }
-}
-
-__global__ void __launch_bounds__(kThreads, 2) adam8_step_kernel(const Tile* __restrict__ tiles, int64_t n_tiles,
-                                                              int64_t bucket, float* master, uint16_t* param,
-                                                              const uint16_t* __restrict__ grad, int8_t* mq,
-                                                              uint8_t* vq, float2* scales, int64_t n_blocks,
-                                                              StepC c, int32_t* status) {
-    if ((int64_t)blockIdx.x >= n_tiles) return;
-    const Tile t = tiles[blockIdx.x];
-    // Bounds of the table entry against the bucket; a bad entry is reported,
-    // never accessed.
-    if (t.e0 < 0 || t.n < 0 || t.e0 + t.n > bucket ||
-        (t.kind != TILE_ZERO && (t.blk0 < 0 || t.blk0 + t.nblk > n_blocks)) ||
-        (t.kind == TILE_WHOLE && (t.b <= 0 || t.nblk > kMaxBlk || (t.e0 & (kAlign - 1)) + t.n > kTile))) {
-        if (threadIdx.x == 0) set_status(status, 2);
-        return;
-    }
-    if (t.kind == TILE_WHOLE)
-        whole_tile(t, master, param, grad, mq, vq, scales, c);
-    else if (t.kind == TILE_LARGE)
-        large_block(t, master, param, grad, mq, vq, scales, c);
-    else
-        zero_tile(t, param);
-}
-
-// ------------------------------------------------------- copy-in (TMA bulk)
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void fence_barrier_init() {
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-__device__ __forceinline__ uint64_t global_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-    return t;
-}
-
-// Wait for an mbarrier phase, giving up after ~limit_ns; false on time-out.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
-    const uint64_t t0 = global_ns();
-    for (uint32_t it = 0;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 255u) == 255u && global_ns() - t0 > limit_ns) return false;
-    }
-}
-
-constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s: far beyond any copy
-
-__global__ void __launch_bounds__(kPackThreads) pack_kernel(PackPtrs ptrs, const PackChunk* __restrict__ chunks,
-                                                            int64_t first_chunk, int32_t tensor_base,
-                                                            uint16_t* grad, int64_t bucket, float scale,
-                                                            int32_t* status) {
-    extern __shared__ __align__(128) uint4 sbuf[];
-    __shared__ __align__(8) uint64_t bar;
-    const PackChunk ch = chunks[first_chunk + blockIdx.x];
-    const int32_t ti = ch.tensor - tensor_base;
-    if (ti < 0 || ti >= kMaxPackPtrs || ch.count < 0 || ch.count > kPackChunk || ch.dst_off < 0 ||
-        ch.dst_off + ch.count > bucket) {
-        if (threadIdx.x == 0) set_status(status, 2);
-        return;
-    }
-    const uint16_t* src = ptrs.p[ti] + ch.src_off;
-    uint16_t* dst = grad + ch.dst_off;
-    // Whole 16-byte granules go through one bulk copy into shared memory.
-    const bool aligned = (reinterpret_cast<uintptr_t>(src) & 15u) == 0;
-    const int32_t nbulk = aligned ? (ch.count & ~7) : 0;
-    if (threadIdx.x == 0) {
-        mbar_init(&bar, 1);
-        fence_barrier_init();
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        mbar_arrive_expect_tx(&bar, (uint32_t)nbulk * 2u);
-        if (nbulk > 0) bulk_g2s(sbuf, src, (uint32_t)nbulk * 2u, &bar);
-    }
-    // Scalar tail while the bulk copy is in flight.
-    for (int32_t i = nbulk + threadIdx.x; i < ch.count; i += kPackThreads) {
-        const float f = __fmul_rn(bf16_bits_to_f32(src[i]), scale);
-        dst[i] = __bfloat16_as_ushort(__float2bfloat16_rn(f));
-    }
-    if (!mbar_wait_bounded(&bar, 0, kWaitNs)) {
-        if (threadIdx.x == 0) set_status(status, 1);
-        // Let the copy land before the CTA (and its shared memory) goes away.
-        mbar_wait_bounded(&bar, 0, kWaitNs);
-        return;
-    }
-    for (int32_t v = threadIdx.x; v < nbulk / 8; v += kPackThreads) {
-        const uint4 w = sbuf[v];
-        const uint32_t in[4] = {w.x, w.y, w.z, w.w};
-        uint32_t out[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float lo_f = __fmul_rn(bf16_bits_to_f32(in[q] & 0xffffu), scale);
-            const float hi_f = __fmul_rn(bf16_bits_to_f32(in[q] >> 16), scale);
-            out[q] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo_f)) |
-                     ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi_f)) << 16);
-        }
-        __stcs(reinterpret_cast<uint4*>(dst) + v, make_uint4(out[0], out[1], out[2], out[3]));
-    }
-}
+using namespace dbuf_k;
 
 StepC make_step_constants(const dbuf_adam_hparams& hp, float grad_scale) {
     const double B1 = hp.beta1, B2 = hp.beta2, lr = hp.lr, wd = hp.weight_decay, eps = hp.eps;
@@ -782,6 +181,24 @@ dbuf_status check_device(const dbuf_t* db, const char* who) {
     if (dev != db->device)
         return fail(DBUF_EINVAL, std::string(who) + ": current device " + std::to_string(dev) +
                                      " is not the dbuf's device " + std::to_string(db->device));
+    return DBUF_OK;
+}
+
+// Persistent grid of the step kernel on the current device: as many CTAs as
+// fit at once (two per SM with its shared-memory ring), never more than tiles.
+dbuf_status step_grid_for(int device, size_t n_tiles, int* grid) {
+    static bool attr_set[64] = {false};
+    if (device >= 0 && device < 64 && !attr_set[device]) {
+        CUDA_TRY(cudaFuncSetAttribute(adam8_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kStepSmem),
+                 "dbuf_create: step kernel shared memory");
+        attr_set[device] = true;
+    }
+    int sms = 0, per_sm = 0;
+    CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device), "dbuf_create: SM count");
+    CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, adam8_step_kernel, kStepThreads, kStepSmem),
+             "dbuf_create: step kernel occupancy");
+    if (per_sm < 1) return fail(DBUF_ECUDA, "dbuf_create: the step kernel does not fit on this device");
+    *grid = (int)std::min<size_t>(n_tiles, (size_t)sms * (size_t)per_sm);
     return DBUF_OK;
 }
 
@@ -831,6 +248,13 @@ extern "C" dbuf_status dbuf_create(const dbuf_plan_t* plan, void* device_base, s
     if (e != cudaSuccess) {
         delete db;
         return fail(DBUF_ECUDA, std::string("dbuf_create: cudaGetDevice: ") + cudaGetErrorString(e));
+    }
+    {
+        dbuf_status gs = step_grid_for(db->device, db->h_tiles.size(), &db->step_grid);
+        if (gs != DBUF_OK) {
+            delete db;
+            return gs;
+        }
     }
     if (device_base) {
         if ((reinterpret_cast<uintptr_t>(device_base) & 255u) != 0 || base_bytes < db->bytes) {
@@ -926,7 +350,7 @@ extern "C" dbuf_status dbuf_adam8_step(dbuf_t* db, const dbuf_adam_hparams* hp, 
     if (db->h_tiles.empty()) return DBUF_OK;
     const StepC c = make_step_constants(*hp, grad_scale);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    adam8_step_kernel<<<(unsigned)db->h_tiles.size(), kThreads, 0, st>>>(
+    adam8_step_kernel<<<(unsigned)db->step_grid, kStepThreads, kStepSmem, st>>>(
         db->tiles, (int64_t)db->h_tiles.size(), db->plan.bucket, db->master, db->param, db->grad, db->mq, db->vq,
         db->scales, db->plan.n_blocks, c, db->status);
     CUDA_TRY(cudaGetLastError(), "dbuf_adam8_step: launch");

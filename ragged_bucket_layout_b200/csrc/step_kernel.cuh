@@ -1,0 +1,624 @@
+// Fused block-wise 8-bit Adam step over a whole ragged bucket (sm_100a).
+//
+// veScale-FSDP (8-bit Adam case study, paper Sec. 6.3; DBuffer group
+// operations, Sec. 5): the quantisation blocks are aligned with the shards,
+// so every block is updated and requantised on its own, and the whole
+// bucket goes through one grouped launch instead of one launch per tensor.
+//
+// Persistent kernel, one CTA per slot (two per SM): 8 consumer warps and one
+// producer warp.  The producer walks the CTA's share of the work table
+// (entries blockIdx.x, blockIdx.x + gridDim.x, ...) and streams each tile's
+// inputs (bf16 grad, fp32 master, int8/uint8 codes, per-block scales) into a
+// 3-stage shared-memory ring with bulk copies (TMA, cp.async.bulk), so the
+// loads of the next tiles are in flight while the consumers compute and wait
+// at barriers.  Consumers read a stage, keep the new m and sqrt(v) of their
+// 16 elements in registers, write weights and the bf16 copy straight to
+// global memory (128-bit stores), reduce each block's absmax, then write the
+// codes.  A LARGE block (longer than a tile) is streamed twice: pass 1
+// updates the weights and finds the absmax; pass 2 reloads grad and the old
+// codes (recently read, so mostly from L2) and recomputes m and sqrt(v)
+// bit-identically to quantise them.
+//
+// Waits on copies are bounded (2 s); a time-out sets status 1 and the CTA
+// drains its own copies before leaving.  One elected consumer thread waits
+// and a named barrier hands the outcome to all consumers, so they agree.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "tables.h"
+#include "tma.cuh"
+
+namespace dbuf_k {
+
+// Per-step scalars (formed on the host in double, rounded to float once).
+// The bias corrections are folded into the step size and eps:
+//   (lr/bc1) m / (sqrt(v)/sqrt(bc2) + eps) = step_hat * m / (sqrt(v) + eps_hat).
+struct StepC {
+    float b1, omb1, b2, omb2, eps_hat, step_hat, decay, gscale;
+};
+
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumers = kConsumerWarps * 32;       // 256 threads
+constexpr int kStepThreads = kConsumers + 32;         // + one producer warp
+constexpr int kStages = 3;
+constexpr int kV = 8;                                 // elements per thread-vector
+constexpr int kHalves = kTile / (kConsumers * kV);    // vectors per thread per tile (2)
+constexpr int kOffG = 0;                              // bf16 grad
+constexpr int kOffP = kOffG + kTile * 2;              // fp32 master
+constexpr int kOffMQ = kOffP + kTile * 4;             // int8 codes of m
+constexpr int kOffVQ = kOffMQ + kTile;                // uint8 codes of sqrt(v)
+constexpr int kOffS = kOffVQ + kTile;                 // float2 scales (<= 256 entries)
+constexpr int kStageBytes = kOffS + 256 * 8;          // 34816
+constexpr int kStepSmem = kStages * kStageBytes;
+constexpr uint32_t kBarCons = 1;                      // named barrier of the consumers
+static_assert(kHalves * kConsumers * kV == kTile, "tile split");
+static_assert(kMaxBlk + 2 <= 256, "scale copy fits its stage slot");
+
+struct StepShared {
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    uint32_t am[256], ar[256];  // block absmax as float bits
+    float dqm[256], dqv[256];   // dequantisation steps of the old codes
+    float qm[256], qv[256];     // quantisation factors of the new codes
+    float red[2][kConsumerWarps];
+    int32_t go[2];
+};
+
+// ---------------------------------------------------------------- arithmetic
+
+// Code bytes to float without the conversion unit: byte b in the low
+// mantissa bits of 2^23 reads as 2^23 + b; subtracting 2^23 is exact.  int8
+// codes have their sign bit flipped first (b = code + 128).
+__device__ __forceinline__ float ubyte_to_f(uint32_t w, uint32_t sel) {
+    return __fsub_rn(__uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540u | sel)), 8388608.0f);
+}
+__device__ __forceinline__ float sbyte_to_f(uint32_t w_flipped, uint32_t sel) {
+    return __fsub_rn(__uint_as_float(__byte_perm(w_flipped, 0x4B000000u, 0x7540u | sel)), 8388736.0f);
+}
+
+// Round to the nearest integer, ties to even, by adding 1.5*2^23: the sum
+// lies where the float spacing is 1, so the addition itself rounds, and the
+// low byte of the sum's bits is the integer's two's-complement low byte.
+// Valid for |x| < 2^22; codes here have |x| <= 255.
+__device__ __forceinline__ uint32_t rne_low_bits(float x) { return __float_as_uint(__fadd_rn(x, 12582912.0f)); }
+
+__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    return __byte_perm(__byte_perm(a, b, 0x0040u), __byte_perm(c, d, 0x0040u), 0x5410u);
+}
+
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// New m and sqrt(v) of one element, every operation rounded on its own.
+__device__ __forceinline__ void new_m_r(float graw, float qmf, float qvf, float dqm, float dqv, const StepC& c,
+                                        float& m, float& r) {
+    const float g = __fmul_rn(graw, c.gscale);
+    const float mo = __fmul_rn(qmf, dqm);
+    const float so = __fmul_rn(qvf, dqv);
+    const float vo = __fmul_rn(so, so);
+    m = __fadd_rn(__fmul_rn(c.b1, mo), __fmul_rn(c.omb1, g));
+    const float v = __fadd_rn(__fmul_rn(c.b2, vo), __fmul_rn(c.omb2, __fmul_rn(g, g)));
+    r = __fsqrt_rn(v);
+}
+
+__device__ __forceinline__ float new_p(float p, float m, float r, const StepC& c) {
+    const float u = __fdiv_rn(m, __fadd_rn(r, c.eps_hat));
+    return __fsub_rn(__fmul_rn(p, c.decay), __fmul_rn(c.step_hat, u));
+}
+
+// ------------------------------------------------------------ vector I/O
+
+struct In8 {
+    uint32_t g[4];   // bf16 pairs
+    float p[8];
+    uint32_t mq[2];  // int8 codes, sign bits flipped
+    uint32_t vq[2];  // uint8 codes
+};
+
+__device__ __forceinline__ float g_of(const In8& x, int i) {
+    const uint32_t w = x.g[i >> 1];
+    return __uint_as_float((i & 1) ? (w & 0xffff0000u) : (w << 16));
+}
+
+// Inputs of elements [vb, vb+8) from a stage (local index li).  When !FULL
+// only elements in [lo, hi) are taken, the rest read as zero.
+template <bool FULL>
+__device__ __forceinline__ void load8_stage(In8& x, const unsigned char* st, int li, int64_t vb, int64_t lo,
+                                            int64_t hi, bool want_p) {
+    if (FULL) {
+        const uint4 g = *reinterpret_cast<const uint4*>(st + kOffG + 2 * li);
+        x.g[0] = g.x; x.g[1] = g.y; x.g[2] = g.z; x.g[3] = g.w;
+        const uint2 a = *reinterpret_cast<const uint2*>(st + kOffMQ + li);
+        const uint2 b = *reinterpret_cast<const uint2*>(st + kOffVQ + li);
+        x.mq[0] = a.x ^ 0x80808080u; x.mq[1] = a.y ^ 0x80808080u;
+        x.vq[0] = b.x; x.vq[1] = b.y;
+        if (want_p) {
+            const float4 p0 = *reinterpret_cast<const float4*>(st + kOffP + 4 * li);
+            const float4 p1 = *reinterpret_cast<const float4*>(st + kOffP + 4 * li + 16);
+            x.p[0] = p0.x; x.p[1] = p0.y; x.p[2] = p0.z; x.p[3] = p0.w;
+            x.p[4] = p1.x; x.p[5] = p1.y; x.p[6] = p1.z; x.p[7] = p1.w;
+        }
+    } else {
+        const uint16_t* g = reinterpret_cast<const uint16_t*>(st + kOffG);
+        const float* p = reinterpret_cast<const float*>(st + kOffP);
+        const uint8_t* a = st + kOffMQ;
+        const uint8_t* b = st + kOffVQ;
+        uint32_t gw[4] = {0, 0, 0, 0}, aw[2] = {0, 0}, bw[2] = {0, 0};
+#pragma unroll
+        for (int i = 0; i < kV; ++i) {
+            const int64_t e = vb + i;
+            const bool in = (e >= lo && e < hi);
+            x.p[i] = (in && want_p) ? p[li + i] : 0.f;
+            if (in) {
+                gw[i >> 1] |= (uint32_t)g[li + i] << (16 * (i & 1));
+                aw[i >> 2] |= (uint32_t)a[li + i] << (8 * (i & 3));
+                bw[i >> 2] |= (uint32_t)b[li + i] << (8 * (i & 3));
+            }
+        }
+        x.g[0] = gw[0]; x.g[1] = gw[1]; x.g[2] = gw[2]; x.g[3] = gw[3];
+        x.mq[0] = aw[0] ^ 0x80808080u; x.mq[1] = aw[1] ^ 0x80808080u;
+        x.vq[0] = bw[0]; x.vq[1] = bw[1];
+    }
+}
+
+template <bool FULL>
+__device__ __forceinline__ void store_p8(const float* p, int64_t vb, int64_t lo, int64_t hi, float* master,
+                                         uint16_t* param) {
+    const uint4 h = make_uint4(bf16x2_bits(p[0], p[1]), bf16x2_bits(p[2], p[3]), bf16x2_bits(p[4], p[5]),
+                               bf16x2_bits(p[6], p[7]));
+    if (FULL) {
+        __stcs(reinterpret_cast<float4*>(master + vb), make_float4(p[0], p[1], p[2], p[3]));
+        __stcs(reinterpret_cast<float4*>(master + vb) + 1, make_float4(p[4], p[5], p[6], p[7]));
+        __stcs(reinterpret_cast<uint4*>(param + vb), h);
+    } else {
+        const uint32_t hw[4] = {h.x, h.y, h.z, h.w};
+#pragma unroll
+        for (int i = 0; i < kV; ++i) {
+            const int64_t e = vb + i;
+            if (e >= lo && e < hi) {
+                master[e] = p[i];
+                param[e] = (uint16_t)(hw[i >> 1] >> (16 * (i & 1)));
+            }
+        }
+    }
+}
+
+// Codes of 8 elements.  |m*qm| <= 127 and 0 <= r*qv <= 255 hold by
+// construction (qm = 127/max|m| over the same values), so no clamp is needed.
+template <bool FULL>
+__device__ __forceinline__ void store_codes8(const float* m, const float* r, const float* qm, const float* qv,
+                                             int64_t vb, int64_t lo, int64_t hi, int8_t* mq, uint8_t* vq) {
+    uint32_t bm[kV], bv[kV];
+#pragma unroll
+    for (int i = 0; i < kV; ++i) {
+        bm[i] = rne_low_bits(__fmul_rn(m[i], qm[i]));
+        bv[i] = rne_low_bits(__fmul_rn(r[i], qv[i]));
+    }
+    const uint2 cm = make_uint2(pack_low_bytes(bm[0], bm[1], bm[2], bm[3]), pack_low_bytes(bm[4], bm[5], bm[6], bm[7]));
+    const uint2 cv = make_uint2(pack_low_bytes(bv[0], bv[1], bv[2], bv[3]), pack_low_bytes(bv[4], bv[5], bv[6], bv[7]));
+    if (FULL) {
+        __stcs(reinterpret_cast<uint2*>(mq + vb), cm);
+        __stcs(reinterpret_cast<uint2*>(vq + vb), cv);
+    } else {
+#pragma unroll
+        for (int i = 0; i < kV; ++i) {
+            const int64_t e = vb + i;
+            if (e >= lo && e < hi) {
+                mq[e] = (int8_t)(bm[i] & 0xffu);
+                vq[e] = (uint8_t)(bv[i] & 0xffu);
+            }
+        }
+    }
+}
+
+template <bool FULL>
+__device__ __forceinline__ void codes_one(int64_t vb, int64_t lo, int64_t hi, float qm1, float qv1, const float* m,
+                                          const float* r, int8_t* mq, uint8_t* vq) {
+    float qm[kV], qv[kV];
+#pragma unroll
+    for (int i = 0; i < kV; ++i) {
+        qm[i] = qm1;
+        qv[i] = qv1;
+    }
+    store_codes8<FULL>(m, r, qm, qv, vb, lo, hi, mq, vq);
+}
+
+// Phase 1 for a vector inside one block: update, write weights and bf16 copy.
+template <bool FULL>
+__device__ __forceinline__ void phase1_one(const unsigned char* st, int li, int64_t vb, int64_t lo, int64_t hi,
+                                           float dqm, float dqv, const StepC& c, float* master, uint16_t* param,
+                                           float* m, float* r) {
+    In8 x;
+    load8_stage<FULL>(x, st, li, vb, lo, hi, true);
+#pragma unroll
+    for (int i = 0; i < kV; ++i) {
+        new_m_r(g_of(x, i), sbyte_to_f(x.mq[i >> 2], i & 3), ubyte_to_f(x.vq[i >> 2], i & 3), dqm, dqv, c, m[i],
+                r[i]);
+        x.p[i] = new_p(x.p[i], m[i], r[i], c);
+    }
+    store_p8<FULL>(x.p, vb, lo, hi, master, param);
+}
+
+// Pass 2 of a LARGE block: recompute m and sqrt(v), write the codes.
+template <bool FULL>
+__device__ __forceinline__ void pass2_one(const unsigned char* st, int li, int64_t vb, int64_t lo, int64_t hi,
+                                          float dqm, float dqv, float qm, float qv, const StepC& c, int8_t* mq,
+                                          uint8_t* vq) {
+    In8 x;
+    float m[kV], r[kV];
+    load8_stage<FULL>(x, st, li, vb, lo, hi, false);
+#pragma unroll
+    for (int i = 0; i < kV; ++i)
+        new_m_r(g_of(x, i), sbyte_to_f(x.mq[i >> 2], i & 3), ubyte_to_f(x.vq[i >> 2], i & 3), dqm, dqv, c, m[i],
+                r[i]);
+    codes_one<FULL>(vb, lo, hi, qm, qv, m, r, mq, vq);
+}
+
+// A vector spanning several blocks (blocks shorter than 8 elements or off
+// the 8-element grid): per-element block numbers; absmax straight into
+// shared memory.
+__device__ __noinline__ void phase1_mixed(const unsigned char* st, int li, int64_t vb, int64_t lo, int64_t hi,
+                                          uint32_t b, int bf, const StepC& c, float* master, uint16_t* param,
+                                          StepShared& sh, float* m, float* r) {
+    In8 x;
+    load8_stage<false>(x, st, li, vb, lo, hi, true);
+#pragma unroll
+    for (int i = 0; i < kV; ++i) {
+        const int64_t e = vb + i;
+        const int blk = (e < lo || e >= hi) ? bf : (int)((uint32_t)(e - lo) / b);
+        new_m_r(g_of(x, i), sbyte_to_f(x.mq[i >> 2], i & 3), ubyte_to_f(x.vq[i >> 2], i & 3), sh.dqm[blk],
+                sh.dqv[blk], c, m[i], r[i]);
+        x.p[i] = new_p(x.p[i], m[i], r[i], c);
+        atomicMax(&sh.am[blk], __float_as_uint(fabsf(m[i])));
+        atomicMax(&sh.ar[blk], __float_as_uint(r[i]));
+    }
+    store_p8<false>(x.p, vb, lo, hi, master, param);
+}
+
+__device__ __noinline__ void codes_mixed(int64_t vb, int64_t lo, int64_t hi, uint32_t b, int bf,
+                                         const StepShared& sh, const float* m, const float* r, int8_t* mq,
+                                         uint8_t* vq) {
+    float qm[kV], qv[kV];
+#pragma unroll
+    for (int i = 0; i < kV; ++i) {
+        const int64_t e = vb + i;
+        const int blk = (e < lo || e >= hi) ? bf : (int)((uint32_t)(e - lo) / b);
+        qm[i] = sh.qm[blk];
+        qv[i] = sh.qv[blk];
+    }
+    store_codes8<false>(m, r, qm, qv, vb, lo, hi, mq, vq);
+}
+
+// ------------------------------------------------------------- reductions
+
+// Max over lanes sharing `key` (equal keys are contiguous lanes); true on the
+// first lane of each run, which holds the run's maximum.
+__device__ __forceinline__ bool segmented_max(int key, float& a, float& b) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int ok = __shfl_down_sync(0xffffffffu, key, d);
+        const float oa = __shfl_down_sync(0xffffffffu, a, d);
+        const float ob = __shfl_down_sync(0xffffffffu, b, d);
+        if (lane + d < 32 && ok == key) {
+            a = fmaxf(a, oa);
+            b = fmaxf(b, ob);
+        }
+    }
+    const int prev = __shfl_up_sync(0xffffffffu, key, 1);
+    return (lane == 0) || (prev != key);
+}
+
+__device__ __forceinline__ void warp_max2(float& a, float& b) {
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) {
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, d));
+        b = fmaxf(b, __shfl_xor_sync(0xffffffffu, b, d));
+    }
+}
+
+// ------------------------------------------------------------ pipeline
+
+__device__ __forceinline__ bool tile_ok(const Tile& t, int64_t bucket, int64_t n_blocks) {
+    if (t.e0 < 0 || t.n <= 0 || t.e0 + t.n > bucket) return false;
+    if (t.kind == TILE_ZERO) return true;
+    if (t.blk0 < 0 || t.nblk < 1 || t.blk0 + t.nblk > n_blocks) return false;
+    if (t.kind == TILE_WHOLE) return t.b > 0 && t.nblk <= kMaxBlk && (t.e0 & (kAlign - 1)) + t.n <= kTile;
+    return t.kind == TILE_LARGE && t.nblk == 1;
+}
+
+__device__ __forceinline__ int64_t large_chunks(const Tile& t) {
+    const int64_t a0 = t.e0 & ~int64_t(kAlign - 1);
+    return (t.e0 + t.n - a0 + kTile - 1) / kTile;
+}
+
+// Consumers: wait until stage use k has landed.  Thread 0 waits (bounded),
+// the named barrier hands its verdict to every consumer.
+__device__ __forceinline__ bool wait_stage(StepShared& sh, uint32_t k, int32_t* status) {
+    if (threadIdx.x == 0) {
+        const bool ok = mbar_wait_bounded(&sh.full[k % kStages], (k / kStages) & 1u);
+        sh.go[k & 1u] = ok ? 1 : 0;
+        if (!ok) set_status(status, 1);
+    }
+    named_sync(kBarCons, kConsumers);
+    return sh.go[k & 1u] != 0;
+}
+
+// Consumers: this warp is done reading stage use k.
+__device__ __forceinline__ void release_stage(StepShared& sh, uint32_t k) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(&sh.empty[k % kStages]);
+}
+
+__device__ void step_producer(const Tile* __restrict__ tiles, int64_t n_tiles, int64_t bucket, int64_t n_blocks,
+                              const float* master, const uint16_t* grad, const int8_t* mq, const uint8_t* vq,
+                              const float2* scales, unsigned char* stages, StepShared& sh, int32_t* status) {
+    uint32_t k = 0;
+    bool timed_out = false;
+    for (int64_t ti = blockIdx.x; ti < n_tiles && !timed_out; ti += gridDim.x) {
+        const Tile t = tiles[ti];
+        if (!tile_ok(t, bucket, n_blocks) || t.kind == TILE_ZERO) continue;
+        const int64_t a0 = t.e0 & ~int64_t(kAlign - 1);
+        const int64_t hi = t.e0 + t.n;
+        const int passes = t.kind == TILE_WHOLE ? 1 : 2;
+        const int64_t nch = t.kind == TILE_WHOLE ? 1 : large_chunks(t);
+        for (int pass = 0; pass < passes && !timed_out; ++pass) {
+            for (int64_t ch = 0; ch < nch; ++ch) {
+                const uint32_t s = k % kStages;
+                if (k >= kStages && !mbar_wait_bounded(&sh.empty[s], ((k / kStages) - 1u) & 1u)) {
+                    timed_out = true;
+                    break;
+                }
+                unsigned char* st = stages + s * kStageBytes;
+                const int64_t w0 = a0 + ch * kTile;
+                const uint32_t n16 = (uint32_t)((min(hi - w0, (int64_t)kTile) + 15) & ~int64_t(15));
+                uint32_t bytes = n16 * (pass == 0 ? 8u : 4u);
+                int64_t f = 0;
+                uint32_t ns = 0;
+                if (t.kind == TILE_WHOLE) {
+                    f = t.blk0 & ~int64_t(1);
+                    ns = (uint32_t)((t.blk0 + t.nblk - f + 1) & ~int64_t(1));
+                    bytes += ns * 8u;
+                }
+                mbar_arrive_expect_tx(&sh.full[s], bytes);
+                bulk_g2s(st + kOffG, grad + w0, n16 * 2u, &sh.full[s]);
+                if (pass == 0) bulk_g2s(st + kOffP, master + w0, n16 * 4u, &sh.full[s]);
+                bulk_g2s(st + kOffMQ, mq + w0, n16, &sh.full[s]);
+                bulk_g2s(st + kOffVQ, vq + w0, n16, &sh.full[s]);
+                if (ns) bulk_g2s(st + kOffS, scales + f, ns * 8u, &sh.full[s]);
+                ++k;
+            }
+        }
+    }
+    if (timed_out) {
+        set_status(status, 1);
+        // Let the copies already issued land before the CTA can go away.
+        for (uint32_t j = k > (uint32_t)kStages ? k - kStages : 0u; j < k; ++j)
+            mbar_wait_bounded(&sh.full[j % kStages], (j / kStages) & 1u);
+    }
+}
+
+__device__ bool whole_tile(const Tile& t, uint32_t k, unsigned char* stages, StepShared& sh, float* master,
+                           uint16_t* param, int8_t* mq, uint8_t* vq, float2* scales, const StepC& c,
+                           int32_t* status) {
+    if (!wait_stage(sh, k, status)) return false;
+    const int tid = threadIdx.x;
+    const unsigned char* st = stages + (k % kStages) * kStageBytes;
+    const int nb = t.nblk;
+    if (tid < nb) {
+        const float2 sc = reinterpret_cast<const float2*>(st + kOffS)[(t.blk0 & 1) + tid];
+        sh.dqm[tid] = __fdiv_rn(sc.x, 127.f);
+        sh.dqv[tid] = __fdiv_rn(sc.y, 255.f);
+        sh.am[tid] = 0u;
+        sh.ar[tid] = 0u;
+    }
+    named_sync(kBarCons, kConsumers);
+
+    const int64_t a0 = t.e0 & ~int64_t(kAlign - 1);
+    const int64_t lo = t.e0, hi = t.e0 + t.n;
+    const uint32_t b = (uint32_t)t.b;
+    const bool single = nb == 1;
+    float m[kHalves][kV], r[kHalves][kV];
+    float mx[kHalves][kV], rx[kHalves][kV];  // mixed-path copies (passed by address)
+    int bf[kHalves];
+    bool one[kHalves];
+    float am[kHalves], ar[kHalves];
+#pragma unroll
+    for (int h = 0; h < kHalves; ++h) {
+        const int li = h * (kConsumers * kV) + kV * tid;
+        const int64_t vb = a0 + li;
+        const int64_t elo = max(vb, lo), ehi = min(vb + kV, hi);
+        const bool any = elo < ehi;
+        const bool full = (vb >= lo) && (vb + kV <= hi);
+        bf[h] = any ? (single ? 0 : (int)((uint32_t)(elo - lo) / b)) : -1;
+        const int bl = any ? (single ? 0 : (int)((uint32_t)(ehi - 1 - lo) / b)) : -1;
+        one[h] = any && (bf[h] == bl);
+        am[h] = 0.f;
+        ar[h] = 0.f;
+        if (one[h]) {
+            const float dqm = sh.dqm[bf[h]], dqv = sh.dqv[bf[h]];
+            if (full)
+                phase1_one<true>(st, li, vb, lo, hi, dqm, dqv, c, master, param, m[h], r[h]);
+            else
+                phase1_one<false>(st, li, vb, lo, hi, dqm, dqv, c, master, param, m[h], r[h]);
+#pragma unroll
+            for (int i = 0; i < kV; ++i) {
+                am[h] = fmaxf(am[h], fabsf(m[h][i]));
+                ar[h] = fmaxf(ar[h], r[h][i]);
+            }
+        } else if (any) {
+            phase1_mixed(st, li, vb, lo, hi, b, bf[h], c, master, param, sh, mx[h], rx[h]);
+        }
+    }
+    release_stage(sh, k);  // the stage's inputs (scales included) are consumed
+
+    if (single) {
+        float a = fmaxf(am[0], am[1]), q = fmaxf(ar[0], ar[1]);
+        warp_max2(a, q);
+        if ((tid & 31) == 0) {
+            atomicMax(&sh.am[0], __float_as_uint(a));
+            atomicMax(&sh.ar[0], __float_as_uint(q));
+        }
+    } else {
+#pragma unroll
+        for (int h = 0; h < kHalves; ++h) {
+            const int key = one[h] ? bf[h] : -1;
+            if (segmented_max(key, am[h], ar[h]) && key >= 0) {
+                atomicMax(&sh.am[key], __float_as_uint(am[h]));
+                atomicMax(&sh.ar[key], __float_as_uint(ar[h]));
+            }
+        }
+    }
+    named_sync(kBarCons, kConsumers);
+    if (tid < nb) {
+        const float AMm = __uint_as_float(sh.am[tid]), AMr = __uint_as_float(sh.ar[tid]);
+        sh.qm[tid] = AMm > 0.f ? __fdiv_rn(127.f, AMm) : 0.f;
+        sh.qv[tid] = AMr > 0.f ? __fdiv_rn(255.f, AMr) : 0.f;
+        scales[t.blk0 + tid] = make_float2(AMm, AMr);
+    }
+    named_sync(kBarCons, kConsumers);
+#pragma unroll
+    for (int h = 0; h < kHalves; ++h) {
+        const int li = h * (kConsumers * kV) + kV * tid;
+        const int64_t vb = a0 + li;
+        const bool any = max(vb, lo) < min(vb + kV, hi);
+        const bool full = (vb >= lo) && (vb + kV <= hi);
+        if (one[h]) {
+            const float qm = sh.qm[bf[h]], qv = sh.qv[bf[h]];
+            if (full)
+                codes_one<true>(vb, lo, hi, qm, qv, m[h], r[h], mq, vq);
+            else
+                codes_one<false>(vb, lo, hi, qm, qv, m[h], r[h], mq, vq);
+        } else if (any) {
+            codes_mixed(vb, lo, hi, b, bf[h], sh, mx[h], rx[h], mq, vq);
+        }
+    }
+    return true;
+}
+
+__device__ bool large_tile(const Tile& t, uint32_t& k, unsigned char* stages, StepShared& sh, float* master,
+                           uint16_t* param, int8_t* mq, uint8_t* vq, float2* scales, const StepC& c,
+                           int32_t* status) {
+    const int tid = threadIdx.x;
+    const float2 sc = scales[t.blk0];
+    const float dqm = __fdiv_rn(sc.x, 127.f), dqv = __fdiv_rn(sc.y, 255.f);
+    const int64_t a0 = t.e0 & ~int64_t(kAlign - 1);
+    const int64_t lo = t.e0, hi = t.e0 + t.n;
+    const int64_t nch = large_chunks(t);
+
+    float am = 0.f, ar = 0.f;
+    for (int64_t ch = 0; ch < nch; ++ch) {
+        if (!wait_stage(sh, k, status)) return false;
+        const unsigned char* st = stages + (k % kStages) * kStageBytes;
+#pragma unroll
+        for (int h = 0; h < kHalves; ++h) {
+            const int li = h * (kConsumers * kV) + kV * tid;
+            const int64_t vb = a0 + ch * kTile + li;
+            if (vb >= hi || vb + kV <= lo) continue;
+            float m[kV], r[kV];
+            if (vb >= lo && vb + kV <= hi)
+                phase1_one<true>(st, li, vb, lo, hi, dqm, dqv, c, master, param, m, r);
+            else
+                phase1_one<false>(st, li, vb, lo, hi, dqm, dqv, c, master, param, m, r);
+#pragma unroll
+            for (int i = 0; i < kV; ++i) {
+                am = fmaxf(am, fabsf(m[i]));
+                ar = fmaxf(ar, r[i]);
+            }
+        }
+        release_stage(sh, k);
+        ++k;
+    }
+    warp_max2(am, ar);
+    if ((tid & 31) == 0) {
+        sh.red[0][tid >> 5] = am;
+        sh.red[1][tid >> 5] = ar;
+    }
+    named_sync(kBarCons, kConsumers);
+    if (tid == 0) {
+        float a = 0.f, q = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) {
+            a = fmaxf(a, sh.red[0][w]);
+            q = fmaxf(q, sh.red[1][w]);
+        }
+        sh.qm[0] = a > 0.f ? __fdiv_rn(127.f, a) : 0.f;
+        sh.qv[0] = q > 0.f ? __fdiv_rn(255.f, q) : 0.f;
+        scales[t.blk0] = make_float2(a, q);
+    }
+    named_sync(kBarCons, kConsumers);
+    const float qm = sh.qm[0], qv = sh.qv[0];
+    for (int64_t ch = 0; ch < nch; ++ch) {
+        if (!wait_stage(sh, k, status)) return false;
+        const unsigned char* st = stages + (k % kStages) * kStageBytes;
+#pragma unroll
+        for (int h = 0; h < kHalves; ++h) {
+            const int li = h * (kConsumers * kV) + kV * tid;
+            const int64_t vb = a0 + ch * kTile + li;
+            if (vb >= hi || vb + kV <= lo) continue;
+            if (vb >= lo && vb + kV <= hi)
+                pass2_one<true>(st, li, vb, lo, hi, dqm, dqv, qm, qv, c, mq, vq);
+            else
+                pass2_one<false>(st, li, vb, lo, hi, dqm, dqv, qm, qv, c, mq, vq);
+        }
+        release_stage(sh, k);
+        ++k;
+    }
+    return true;
+}
+
+__device__ void zero_tile(const Tile& t, uint16_t* param) {
+    const int64_t lo = t.e0, hi = t.e0 + t.n;
+    const int64_t a0 = t.e0 & ~int64_t(kAlign - 1);
+    for (int64_t vb = a0 + (int64_t)kV * threadIdx.x; vb < hi; vb += (int64_t)kV * kConsumers) {
+        if (vb >= lo && vb + kV <= hi) {
+            __stcs(reinterpret_cast<uint4*>(param + vb), make_uint4(0, 0, 0, 0));
+        } else {
+            for (int i = 0; i < kV; ++i)
+                if (vb + i >= lo && vb + i < hi) param[vb + i] = 0;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kStepThreads, 2)
+    adam8_step_kernel(const Tile* __restrict__ tiles, int64_t n_tiles, int64_t bucket, float* master,
+                      uint16_t* param, const uint16_t* grad, int8_t* mq, uint8_t* vq, float2* scales,
+                      int64_t n_blocks, StepC c, int32_t* status) {
+    extern __shared__ __align__(128) unsigned char stages[];
+    __shared__ StepShared sh;
+    const int tid = threadIdx.x;
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sh.full[s], 1);
+            mbar_init(&sh.empty[s], kConsumerWarps);
+        }
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (tid >= kConsumers) {  // producer warp: one lane issues all copies
+        if (tid == kConsumers)
+            step_producer(tiles, n_tiles, bucket, n_blocks, master, grad, mq, vq, scales, stages, sh, status);
+        return;
+    }
+    uint32_t k = 0;
+    for (int64_t ti = blockIdx.x; ti < n_tiles; ti += gridDim.x) {
+        const Tile t = tiles[ti];
+        if (!tile_ok(t, bucket, n_blocks)) {
+            if (tid == 0) set_status(status, 2);
+            continue;
+        }
+        if (t.kind == TILE_ZERO) {
+            zero_tile(t, param);
+        } else if (t.kind == TILE_WHOLE) {
+            if (!whole_tile(t, k, stages, sh, master, param, mq, vq, scales, c, status)) return;
+            ++k;
+        } else {
+            if (!large_tile(t, k, stages, sh, master, param, mq, vq, scales, c, status)) return;
+        }
+    }
+}
+
+}  // namespace dbuf_k

@@ -1,0 +1,39 @@
+// Work tables shared by the host builder (dbuf.cu) and the kernels.
+#pragma once
+
+#include <cstdint>
+
+namespace dbuf_k {
+
+constexpr int kAlign = 16;             // tensor starts are multiples of 16 elements
+constexpr int kTile = 4096;            // elements per tile / pipeline stage
+constexpr int kMaxBlk = 254;           // whole blocks per WHOLE tile (scales fit one 2 KB copy)
+constexpr int64_t kZeroChunk = 65536;  // elements per ZERO tile
+constexpr int64_t kPackChunk = 16384;  // elements per copy-in CTA (32 KB)
+
+enum : int32_t { TILE_WHOLE = 0, TILE_LARGE = 1, TILE_ZERO = 2 };
+
+// One entry of the step kernel's work table.
+//   WHOLE: up to kMaxBlk whole blocks of one tensor, (e0 % 16) + n <= kTile.
+//   LARGE: one block longer than that, streamed in kTile chunks, twice.
+//   ZERO : a padding range; its bf16 copy is set to zero.
+struct Tile {
+    int64_t e0;    // first bucket element
+    int64_t blk0;  // index of the first block (scale index)
+    int64_t n;     // elements
+    int32_t b;     // block size (WHOLE), 0 otherwise
+    int32_t kind;
+    int32_t nblk;  // blocks in the entry
+    int32_t pad_;
+};
+static_assert(sizeof(Tile) == 40, "tile layout");
+
+// One CTA of the copy-in gather.
+struct PackChunk {
+    int64_t src_off;  // element offset in the source tensor
+    int64_t dst_off;  // element offset in the bucket
+    int32_t tensor;   // caller's tensor index
+    int32_t count;    // elements
+};
+
+}  // namespace dbuf_k

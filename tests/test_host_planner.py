@@ -175,7 +175,7 @@ def test_work_table_covers_bucket_once(name):
         assert t["first_block"] == j
         if t["kind"] == 0:
             b = t["block_elems"]
-            assert 1 <= b <= 4096 and 1 <= t["n_blocks"] <= 256
+            assert 1 <= b <= 4096 and 1 <= t["n_blocks"] <= 254
             assert (e0 % 16) + n <= 4096
             assert np.all(length[j:j + t["n_blocks"] - 1] == b)
             assert int(length[j:j + t["n_blocks"]].sum()) == n
