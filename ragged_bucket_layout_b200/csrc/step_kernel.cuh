@@ -11,9 +11,10 @@
 // inputs (bf16 grad, fp32 master, int8/uint8 codes, per-block scales) into a
 // 3-stage shared-memory ring with bulk copies (TMA, cp.async.bulk), so the
 // loads of the next tiles are in flight while the consumers compute and wait
-// at barriers.  Consumers read a stage, keep the new m and sqrt(v) of their
-// 16 elements in registers, write weights and the bf16 copy straight to
-// global memory (128-bit stores), reduce each block's absmax, then write the
+// at barriers.  Consumers read a stage (16 elements per thread, as four
+// 4-element vectors), write weights and the bf16 copy straight to global
+// memory, put the new m and sqrt(v) back into their own bytes of the stage,
+// reduce each block's absmax, then read m and sqrt(v) back and write the
 // codes.  A LARGE block (longer than a tile) is streamed twice: pass 1
 // updates the weights and finds the absmax; pass 2 reloads grad and the old
 // codes (recently read, so mostly from L2) and recomputes m and sqrt(v)
@@ -42,8 +43,8 @@ constexpr int kConsumerWarps = 8;
 constexpr int kConsumers = kConsumerWarps * 32;       // 256 threads
 constexpr int kStepThreads = kConsumers + 32;         // + one producer warp
 constexpr int kStages = 3;
-constexpr int kV = 8;                                 // elements per thread-vector
-constexpr int kHalves = kTile / (kConsumers * kV);    // vectors per thread per tile (2)
+constexpr int kV = 4;                                 // elements per thread-vector
+constexpr int kSub = kTile / (kConsumers * kV);       // vectors per thread per tile (4)
 constexpr int kOffG = 0;                              // bf16 grad
 constexpr int kOffP = kOffG + kTile * 2;              // fp32 master
 constexpr int kOffMQ = kOffP + kTile * 4;             // int8 codes of m
@@ -52,7 +53,7 @@ constexpr int kOffS = kOffVQ + kTile;                 // float2 scales (<= 256 e
 constexpr int kStageBytes = kOffS + 256 * 8;          // 34816
 constexpr int kStepSmem = kStages * kStageBytes;
 constexpr uint32_t kBarCons = 1;                      // named barrier of the consumers
-static_assert(kHalves * kConsumers * kV == kTile, "tile split");
+static_assert(kSub * kConsumers * kV == kTile, "tile split");
 static_assert(kMaxBlk + 2 <= 256, "scale copy fits its stage slot");
 
 struct StepShared {
@@ -110,43 +111,43 @@ __device__ __forceinline__ float new_p(float p, float m, float r, const StepC& c
 }
 
 // ------------------------------------------------------------ vector I/O
+//
+// Thread-vector = 4 consecutive elements at local index li (a multiple of 4)
+// of a stage.  Its bytes in the stage: grad [2li, 2li+8), master
+// [4li, 4li+16), codes [li, li+4) twice.  After phase 1 the thread's new m
+// goes to its master bytes and its new sqrt(v) to its grad (2 values) and
+// code bytes (1 + 1 values): 16 + 16 bytes that no other thread touches.
 
-struct In8 {
-    uint32_t g[4];   // bf16 pairs
-    float p[8];
-    uint32_t mq[2];  // int8 codes, sign bits flipped
-    uint32_t vq[2];  // uint8 codes
+struct In4 {
+    uint32_t g[2];  // bf16 pairs
+    float p[4];
+    uint32_t mq;    // int8 codes, sign bits flipped
+    uint32_t vq;    // uint8 codes
 };
 
-__device__ __forceinline__ float g_of(const In8& x, int i) {
+__device__ __forceinline__ float g_of(const In4& x, int i) {
     const uint32_t w = x.g[i >> 1];
     return __uint_as_float((i & 1) ? (w & 0xffff0000u) : (w << 16));
 }
 
-// Inputs of elements [vb, vb+8) from a stage (local index li).  When !FULL
-// only elements in [lo, hi) are taken, the rest read as zero.
+// When !FULL only elements in [lo, hi) are taken; the rest read as zero.
 template <bool FULL>
-__device__ __forceinline__ void load8_stage(In8& x, const unsigned char* st, int li, int64_t vb, int64_t lo,
-                                            int64_t hi, bool want_p) {
+__device__ __forceinline__ void load4(In4& x, const unsigned char* st, int li, int64_t vb, int64_t lo, int64_t hi,
+                                      bool want_p) {
     if (FULL) {
-        const uint4 g = *reinterpret_cast<const uint4*>(st + kOffG + 2 * li);
-        x.g[0] = g.x; x.g[1] = g.y; x.g[2] = g.z; x.g[3] = g.w;
-        const uint2 a = *reinterpret_cast<const uint2*>(st + kOffMQ + li);
-        const uint2 b = *reinterpret_cast<const uint2*>(st + kOffVQ + li);
-        x.mq[0] = a.x ^ 0x80808080u; x.mq[1] = a.y ^ 0x80808080u;
-        x.vq[0] = b.x; x.vq[1] = b.y;
+        const uint2 g = *reinterpret_cast<const uint2*>(st + kOffG + 2 * li);
+        x.g[0] = g.x;
+        x.g[1] = g.y;
+        x.mq = *reinterpret_cast<const uint32_t*>(st + kOffMQ + li) ^ 0x80808080u;
+        x.vq = *reinterpret_cast<const uint32_t*>(st + kOffVQ + li);
         if (want_p) {
-            const float4 p0 = *reinterpret_cast<const float4*>(st + kOffP + 4 * li);
-            const float4 p1 = *reinterpret_cast<const float4*>(st + kOffP + 4 * li + 16);
-            x.p[0] = p0.x; x.p[1] = p0.y; x.p[2] = p0.z; x.p[3] = p0.w;
-            x.p[4] = p1.x; x.p[5] = p1.y; x.p[6] = p1.z; x.p[7] = p1.w;
+            const float4 p = *reinterpret_cast<const float4*>(st + kOffP + 4 * li);
+            x.p[0] = p.x; x.p[1] = p.y; x.p[2] = p.z; x.p[3] = p.w;
         }
     } else {
         const uint16_t* g = reinterpret_cast<const uint16_t*>(st + kOffG);
         const float* p = reinterpret_cast<const float*>(st + kOffP);
-        const uint8_t* a = st + kOffMQ;
-        const uint8_t* b = st + kOffVQ;
-        uint32_t gw[4] = {0, 0, 0, 0}, aw[2] = {0, 0}, bw[2] = {0, 0};
+        uint32_t gw[2] = {0, 0}, a = 0, b = 0;
 #pragma unroll
         for (int i = 0; i < kV; ++i) {
             const int64_t e = vb + i;
@@ -154,42 +155,57 @@ __device__ __forceinline__ void load8_stage(In8& x, const unsigned char* st, int
             x.p[i] = (in && want_p) ? p[li + i] : 0.f;
             if (in) {
                 gw[i >> 1] |= (uint32_t)g[li + i] << (16 * (i & 1));
-                aw[i >> 2] |= (uint32_t)a[li + i] << (8 * (i & 3));
-                bw[i >> 2] |= (uint32_t)b[li + i] << (8 * (i & 3));
+                a |= (uint32_t)st[kOffMQ + li + i] << (8 * i);
+                b |= (uint32_t)st[kOffVQ + li + i] << (8 * i);
             }
         }
-        x.g[0] = gw[0]; x.g[1] = gw[1]; x.g[2] = gw[2]; x.g[3] = gw[3];
-        x.mq[0] = aw[0] ^ 0x80808080u; x.mq[1] = aw[1] ^ 0x80808080u;
-        x.vq[0] = bw[0]; x.vq[1] = bw[1];
+        x.g[0] = gw[0];
+        x.g[1] = gw[1];
+        x.mq = a ^ 0x80808080u;
+        x.vq = b;
     }
 }
 
+__device__ __forceinline__ void stash_mr(unsigned char* st, int li, const float* m, const float* r) {
+    *reinterpret_cast<float4*>(st + kOffP + 4 * li) = make_float4(m[0], m[1], m[2], m[3]);
+    *reinterpret_cast<uint2*>(st + kOffG + 2 * li) = make_uint2(__float_as_uint(r[0]), __float_as_uint(r[1]));
+    *reinterpret_cast<float*>(st + kOffMQ + li) = r[2];
+    *reinterpret_cast<float*>(st + kOffVQ + li) = r[3];
+}
+
+__device__ __forceinline__ void unstash_mr(const unsigned char* st, int li, float* m, float* r) {
+    const float4 a = *reinterpret_cast<const float4*>(st + kOffP + 4 * li);
+    const uint2 b = *reinterpret_cast<const uint2*>(st + kOffG + 2 * li);
+    m[0] = a.x; m[1] = a.y; m[2] = a.z; m[3] = a.w;
+    r[0] = __uint_as_float(b.x);
+    r[1] = __uint_as_float(b.y);
+    r[2] = *reinterpret_cast<const float*>(st + kOffMQ + li);
+    r[3] = *reinterpret_cast<const float*>(st + kOffVQ + li);
+}
+
 template <bool FULL>
-__device__ __forceinline__ void store_p8(const float* p, int64_t vb, int64_t lo, int64_t hi, float* master,
+__device__ __forceinline__ void store_p4(const float* p, int64_t vb, int64_t lo, int64_t hi, float* master,
                                          uint16_t* param) {
-    const uint4 h = make_uint4(bf16x2_bits(p[0], p[1]), bf16x2_bits(p[2], p[3]), bf16x2_bits(p[4], p[5]),
-                               bf16x2_bits(p[6], p[7]));
+    const uint2 h = make_uint2(bf16x2_bits(p[0], p[1]), bf16x2_bits(p[2], p[3]));
     if (FULL) {
         __stcs(reinterpret_cast<float4*>(master + vb), make_float4(p[0], p[1], p[2], p[3]));
-        __stcs(reinterpret_cast<float4*>(master + vb) + 1, make_float4(p[4], p[5], p[6], p[7]));
-        __stcs(reinterpret_cast<uint4*>(param + vb), h);
+        __stcs(reinterpret_cast<uint2*>(param + vb), h);
     } else {
-        const uint32_t hw[4] = {h.x, h.y, h.z, h.w};
 #pragma unroll
         for (int i = 0; i < kV; ++i) {
             const int64_t e = vb + i;
             if (e >= lo && e < hi) {
                 master[e] = p[i];
-                param[e] = (uint16_t)(hw[i >> 1] >> (16 * (i & 1)));
+                param[e] = (uint16_t)(((i < 2) ? h.x : h.y) >> (16 * (i & 1)));
             }
         }
     }
 }
 
-// Codes of 8 elements.  |m*qm| <= 127 and 0 <= r*qv <= 255 hold by
+// Codes of 4 elements.  |m*qm| <= 127 and 0 <= r*qv <= 255 hold by
 // construction (qm = 127/max|m| over the same values), so no clamp is needed.
 template <bool FULL>
-__device__ __forceinline__ void store_codes8(const float* m, const float* r, const float* qm, const float* qv,
+__device__ __forceinline__ void store_codes4(const float* m, const float* r, const float* qm, const float* qv,
                                              int64_t vb, int64_t lo, int64_t hi, int8_t* mq, uint8_t* vq) {
     uint32_t bm[kV], bv[kV];
 #pragma unroll
@@ -197,11 +213,9 @@ __device__ __forceinline__ void store_codes8(const float* m, const float* r, con
         bm[i] = rne_low_bits(__fmul_rn(m[i], qm[i]));
         bv[i] = rne_low_bits(__fmul_rn(r[i], qv[i]));
     }
-    const uint2 cm = make_uint2(pack_low_bytes(bm[0], bm[1], bm[2], bm[3]), pack_low_bytes(bm[4], bm[5], bm[6], bm[7]));
-    const uint2 cv = make_uint2(pack_low_bytes(bv[0], bv[1], bv[2], bv[3]), pack_low_bytes(bv[4], bv[5], bv[6], bv[7]));
     if (FULL) {
-        __stcs(reinterpret_cast<uint2*>(mq + vb), cm);
-        __stcs(reinterpret_cast<uint2*>(vq + vb), cv);
+        __stcs(reinterpret_cast<uint32_t*>(mq + vb), pack_low_bytes(bm[0], bm[1], bm[2], bm[3]));
+        __stcs(reinterpret_cast<uint32_t*>(vq + vb), pack_low_bytes(bv[0], bv[1], bv[2], bv[3]));
     } else {
 #pragma unroll
         for (int i = 0; i < kV; ++i) {
@@ -214,82 +228,19 @@ __device__ __forceinline__ void store_codes8(const float* m, const float* r, con
     }
 }
 
+// Update of one vector whose elements share dqm/dqv (one block).
 template <bool FULL>
-__device__ __forceinline__ void codes_one(int64_t vb, int64_t lo, int64_t hi, float qm1, float qv1, const float* m,
-                                          const float* r, int8_t* mq, uint8_t* vq) {
-    float qm[kV], qv[kV];
+__device__ __forceinline__ void update4(const unsigned char* st, int li, int64_t vb, int64_t lo, int64_t hi,
+                                        float dqm, float dqv, const StepC& c, float* master, uint16_t* param,
+                                        float* m, float* r) {
+    In4 x;
+    load4<FULL>(x, st, li, vb, lo, hi, true);
 #pragma unroll
     for (int i = 0; i < kV; ++i) {
-        qm[i] = qm1;
-        qv[i] = qv1;
-    }
-    store_codes8<FULL>(m, r, qm, qv, vb, lo, hi, mq, vq);
-}
-
-// Phase 1 for a vector inside one block: update, write weights and bf16 copy.
-template <bool FULL>
-__device__ __forceinline__ void phase1_one(const unsigned char* st, int li, int64_t vb, int64_t lo, int64_t hi,
-                                           float dqm, float dqv, const StepC& c, float* master, uint16_t* param,
-                                           float* m, float* r) {
-    In8 x;
-    load8_stage<FULL>(x, st, li, vb, lo, hi, true);
-#pragma unroll
-    for (int i = 0; i < kV; ++i) {
-        new_m_r(g_of(x, i), sbyte_to_f(x.mq[i >> 2], i & 3), ubyte_to_f(x.vq[i >> 2], i & 3), dqm, dqv, c, m[i],
-                r[i]);
+        new_m_r(g_of(x, i), sbyte_to_f(x.mq, i), ubyte_to_f(x.vq, i), dqm, dqv, c, m[i], r[i]);
         x.p[i] = new_p(x.p[i], m[i], r[i], c);
     }
-    store_p8<FULL>(x.p, vb, lo, hi, master, param);
-}
-
-// Pass 2 of a LARGE block: recompute m and sqrt(v), write the codes.
-template <bool FULL>
-__device__ __forceinline__ void pass2_one(const unsigned char* st, int li, int64_t vb, int64_t lo, int64_t hi,
-                                          float dqm, float dqv, float qm, float qv, const StepC& c, int8_t* mq,
-                                          uint8_t* vq) {
-    In8 x;
-    float m[kV], r[kV];
-    load8_stage<FULL>(x, st, li, vb, lo, hi, false);
-#pragma unroll
-    for (int i = 0; i < kV; ++i)
-        new_m_r(g_of(x, i), sbyte_to_f(x.mq[i >> 2], i & 3), ubyte_to_f(x.vq[i >> 2], i & 3), dqm, dqv, c, m[i],
-                r[i]);
-    codes_one<FULL>(vb, lo, hi, qm, qv, m, r, mq, vq);
-}
-
-// A vector spanning several blocks (blocks shorter than 8 elements or off
-// the 8-element grid): per-element block numbers; absmax straight into
-// shared memory.
-__device__ __noinline__ void phase1_mixed(const unsigned char* st, int li, int64_t vb, int64_t lo, int64_t hi,
-                                          uint32_t b, int bf, const StepC& c, float* master, uint16_t* param,
-                                          StepShared& sh, float* m, float* r) {
-    In8 x;
-    load8_stage<false>(x, st, li, vb, lo, hi, true);
-#pragma unroll
-    for (int i = 0; i < kV; ++i) {
-        const int64_t e = vb + i;
-        const int blk = (e < lo || e >= hi) ? bf : (int)((uint32_t)(e - lo) / b);
-        new_m_r(g_of(x, i), sbyte_to_f(x.mq[i >> 2], i & 3), ubyte_to_f(x.vq[i >> 2], i & 3), sh.dqm[blk],
-                sh.dqv[blk], c, m[i], r[i]);
-        x.p[i] = new_p(x.p[i], m[i], r[i], c);
-        atomicMax(&sh.am[blk], __float_as_uint(fabsf(m[i])));
-        atomicMax(&sh.ar[blk], __float_as_uint(r[i]));
-    }
-    store_p8<false>(x.p, vb, lo, hi, master, param);
-}
-
-__device__ __noinline__ void codes_mixed(int64_t vb, int64_t lo, int64_t hi, uint32_t b, int bf,
-                                         const StepShared& sh, const float* m, const float* r, int8_t* mq,
-                                         uint8_t* vq) {
-    float qm[kV], qv[kV];
-#pragma unroll
-    for (int i = 0; i < kV; ++i) {
-        const int64_t e = vb + i;
-        const int blk = (e < lo || e >= hi) ? bf : (int)((uint32_t)(e - lo) / b);
-        qm[i] = sh.qm[blk];
-        qv[i] = sh.qv[blk];
-    }
-    store_codes8<false>(m, r, qm, qv, vb, lo, hi, mq, vq);
+    store_p4<FULL>(x.p, vb, lo, hi, master, param);
 }
 
 // ------------------------------------------------------------- reductions
@@ -320,6 +271,22 @@ __device__ __forceinline__ void warp_max2(float& a, float& b) {
     }
 }
 
+// Fold (a, b) of every lane into block `key` of shared memory (key < 0: no
+// contribution).  One atomic per warp when the whole warp is in one block.
+__device__ __forceinline__ void block_max_to_smem(int key, float a, float b, StepShared& sh) {
+    const int k0 = __shfl_sync(0xffffffffu, key, 0);
+    if (__all_sync(0xffffffffu, key == k0)) {
+        warp_max2(a, b);
+        if ((threadIdx.x & 31) == 0 && k0 >= 0) {
+            atomicMax(&sh.am[k0], __float_as_uint(a));
+            atomicMax(&sh.ar[k0], __float_as_uint(b));
+        }
+    } else if (segmented_max(key, a, b) && key >= 0) {
+        atomicMax(&sh.am[key], __float_as_uint(a));
+        atomicMax(&sh.ar[key], __float_as_uint(b));
+    }
+}
+
 // ------------------------------------------------------------ pipeline
 
 __device__ __forceinline__ bool tile_ok(const Tile& t, int64_t bucket, int64_t n_blocks) {
@@ -347,7 +314,7 @@ __device__ __forceinline__ bool wait_stage(StepShared& sh, uint32_t k, int32_t* 
     return sh.go[k & 1u] != 0;
 }
 
-// Consumers: this warp is done reading stage use k.
+// Consumers: this warp is done with stage use k.
 __device__ __forceinline__ void release_stage(StepShared& sh, uint32_t k) {
     __syncwarp();
     if ((threadIdx.x & 31) == 0) mbar_arrive(&sh.empty[k % kStages]);
@@ -401,12 +368,14 @@ __device__ void step_producer(const Tile* __restrict__ tiles, int64_t n_tiles, i
     }
 }
 
+// Whole blocks: phase 1 updates the weights and stashes m, sqrt(v) in the
+// stage; block maxima meet in shared memory; phase 2 writes the codes.
 __device__ bool whole_tile(const Tile& t, uint32_t k, unsigned char* stages, StepShared& sh, float* master,
                            uint16_t* param, int8_t* mq, uint8_t* vq, float2* scales, const StepC& c,
                            int32_t* status) {
     if (!wait_stage(sh, k, status)) return false;
     const int tid = threadIdx.x;
-    const unsigned char* st = stages + (k % kStages) * kStageBytes;
+    unsigned char* st = stages + (k % kStages) * kStageBytes;
     const int nb = t.nblk;
     if (tid < nb) {
         const float2 sc = reinterpret_cast<const float2*>(st + kOffS)[(t.blk0 & 1) + tid];
@@ -421,57 +390,54 @@ __device__ bool whole_tile(const Tile& t, uint32_t k, unsigned char* stages, Ste
     const int64_t lo = t.e0, hi = t.e0 + t.n;
     const uint32_t b = (uint32_t)t.b;
     const bool single = nb == 1;
-    float m[kHalves][kV], r[kHalves][kV];
-    float mx[kHalves][kV], rx[kHalves][kV];  // mixed-path copies (passed by address)
-    int bf[kHalves];
-    bool one[kHalves];
-    float am[kHalves], ar[kHalves];
+    float am1 = 0.f, ar1 = 0.f;  // single block: running max over the thread's vectors
 #pragma unroll
-    for (int h = 0; h < kHalves; ++h) {
-        const int li = h * (kConsumers * kV) + kV * tid;
+    for (int j = 0; j < kSub; ++j) {
+        const int li = j * (kConsumers * kV) + kV * tid;
         const int64_t vb = a0 + li;
         const int64_t elo = max(vb, lo), ehi = min(vb + kV, hi);
         const bool any = elo < ehi;
         const bool full = (vb >= lo) && (vb + kV <= hi);
-        bf[h] = any ? (single ? 0 : (int)((uint32_t)(elo - lo) / b)) : -1;
+        const int bf = any ? (single ? 0 : (int)((uint32_t)(elo - lo) / b)) : -1;
         const int bl = any ? (single ? 0 : (int)((uint32_t)(ehi - 1 - lo) / b)) : -1;
-        one[h] = any && (bf[h] == bl);
-        am[h] = 0.f;
-        ar[h] = 0.f;
-        if (one[h]) {
-            const float dqm = sh.dqm[bf[h]], dqv = sh.dqv[bf[h]];
+        float m[kV], r[kV];
+        float am = 0.f, ar = 0.f;
+        if (any && bf == bl) {
             if (full)
-                phase1_one<true>(st, li, vb, lo, hi, dqm, dqv, c, master, param, m[h], r[h]);
+                update4<true>(st, li, vb, lo, hi, sh.dqm[bf], sh.dqv[bf], c, master, param, m, r);
             else
-                phase1_one<false>(st, li, vb, lo, hi, dqm, dqv, c, master, param, m[h], r[h]);
+                update4<false>(st, li, vb, lo, hi, sh.dqm[bf], sh.dqv[bf], c, master, param, m, r);
 #pragma unroll
             for (int i = 0; i < kV; ++i) {
-                am[h] = fmaxf(am[h], fabsf(m[h][i]));
-                ar[h] = fmaxf(ar[h], r[h][i]);
+                am = fmaxf(am, fabsf(m[i]));
+                ar = fmaxf(ar, r[i]);
             }
+            stash_mr(st, li, m, r);
         } else if (any) {
-            phase1_mixed(st, li, vb, lo, hi, b, bf[h], c, master, param, sh, mx[h], rx[h]);
-        }
-    }
-    release_stage(sh, k);  // the stage's inputs (scales included) are consumed
-
-    if (single) {
-        float a = fmaxf(am[0], am[1]), q = fmaxf(ar[0], ar[1]);
-        warp_max2(a, q);
-        if ((tid & 31) == 0) {
-            atomicMax(&sh.am[0], __float_as_uint(a));
-            atomicMax(&sh.ar[0], __float_as_uint(q));
-        }
-    } else {
+            // blocks shorter than a vector or off the 4-element grid
+            In4 x;
+            load4<false>(x, st, li, vb, lo, hi, true);
 #pragma unroll
-        for (int h = 0; h < kHalves; ++h) {
-            const int key = one[h] ? bf[h] : -1;
-            if (segmented_max(key, am[h], ar[h]) && key >= 0) {
-                atomicMax(&sh.am[key], __float_as_uint(am[h]));
-                atomicMax(&sh.ar[key], __float_as_uint(ar[h]));
+            for (int i = 0; i < kV; ++i) {
+                const int64_t e = vb + i;
+                const int blk = (e < lo || e >= hi) ? bf : (int)((uint32_t)(e - lo) / b);
+                new_m_r(g_of(x, i), sbyte_to_f(x.mq, i), ubyte_to_f(x.vq, i), sh.dqm[blk], sh.dqv[blk], c, m[i],
+                        r[i]);
+                x.p[i] = new_p(x.p[i], m[i], r[i], c);
+                atomicMax(&sh.am[blk], __float_as_uint(fabsf(m[i])));
+                atomicMax(&sh.ar[blk], __float_as_uint(r[i]));
             }
+            store_p4<false>(x.p, vb, lo, hi, master, param);
+            stash_mr(st, li, m, r);
+        }
+        if (single) {
+            am1 = fmaxf(am1, am);
+            ar1 = fmaxf(ar1, ar);
+        } else {
+            block_max_to_smem((any && bf == bl) ? bf : -1, am, ar, sh);
         }
     }
+    if (single) block_max_to_smem(0, am1, ar1, sh);
     named_sync(kBarCons, kConsumers);
     if (tid < nb) {
         const float AMm = __uint_as_float(sh.am[tid]), AMr = __uint_as_float(sh.ar[tid]);
@@ -481,24 +447,35 @@ __device__ bool whole_tile(const Tile& t, uint32_t k, unsigned char* stages, Ste
     }
     named_sync(kBarCons, kConsumers);
 #pragma unroll
-    for (int h = 0; h < kHalves; ++h) {
-        const int li = h * (kConsumers * kV) + kV * tid;
+    for (int j = 0; j < kSub; ++j) {
+        const int li = j * (kConsumers * kV) + kV * tid;
         const int64_t vb = a0 + li;
-        const bool any = max(vb, lo) < min(vb + kV, hi);
+        const int64_t elo = max(vb, lo), ehi = min(vb + kV, hi);
+        if (elo >= ehi) continue;
         const bool full = (vb >= lo) && (vb + kV <= hi);
-        if (one[h]) {
-            const float qm = sh.qm[bf[h]], qv = sh.qv[bf[h]];
-            if (full)
-                codes_one<true>(vb, lo, hi, qm, qv, m[h], r[h], mq, vq);
-            else
-                codes_one<false>(vb, lo, hi, qm, qv, m[h], r[h], mq, vq);
-        } else if (any) {
-            codes_mixed(vb, lo, hi, b, bf[h], sh, mx[h], rx[h], mq, vq);
+        float m[kV], r[kV], qm[kV], qv[kV];
+        unstash_mr(st, li, m, r);
+        const int bf = single ? 0 : (int)((uint32_t)(elo - lo) / b);
+        const int bl = single ? 0 : (int)((uint32_t)(ehi - 1 - lo) / b);
+#pragma unroll
+        for (int i = 0; i < kV; ++i) {
+            const int64_t e = vb + i;
+            const int blk = (bf == bl || e < lo || e >= hi) ? bf : (int)((uint32_t)(e - lo) / b);
+            qm[i] = sh.qm[blk];
+            qv[i] = sh.qv[blk];
         }
+        if (full)
+            store_codes4<true>(m, r, qm, qv, vb, lo, hi, mq, vq);
+        else
+            store_codes4<false>(m, r, qm, qv, vb, lo, hi, mq, vq);
     }
+    release_stage(sh, k);
     return true;
 }
 
+// A block longer than a tile: pass 1 over its chunks updates the weights and
+// finds the absmax; pass 2 reloads grad and old codes, recomputes m and
+// sqrt(v) and writes the codes.
 __device__ bool large_tile(const Tile& t, uint32_t& k, unsigned char* stages, StepShared& sh, float* master,
                            uint16_t* param, int8_t* mq, uint8_t* vq, float2* scales, const StepC& c,
                            int32_t* status) {
@@ -514,15 +491,15 @@ __device__ bool large_tile(const Tile& t, uint32_t& k, unsigned char* stages, St
         if (!wait_stage(sh, k, status)) return false;
         const unsigned char* st = stages + (k % kStages) * kStageBytes;
 #pragma unroll
-        for (int h = 0; h < kHalves; ++h) {
-            const int li = h * (kConsumers * kV) + kV * tid;
+        for (int j = 0; j < kSub; ++j) {
+            const int li = j * (kConsumers * kV) + kV * tid;
             const int64_t vb = a0 + ch * kTile + li;
             if (vb >= hi || vb + kV <= lo) continue;
             float m[kV], r[kV];
             if (vb >= lo && vb + kV <= hi)
-                phase1_one<true>(st, li, vb, lo, hi, dqm, dqv, c, master, param, m, r);
+                update4<true>(st, li, vb, lo, hi, dqm, dqv, c, master, param, m, r);
             else
-                phase1_one<false>(st, li, vb, lo, hi, dqm, dqv, c, master, param, m, r);
+                update4<false>(st, li, vb, lo, hi, dqm, dqv, c, master, param, m, r);
 #pragma unroll
             for (int i = 0; i < kV; ++i) {
                 am = fmaxf(am, fabsf(m[i]));
@@ -550,19 +527,35 @@ __device__ bool large_tile(const Tile& t, uint32_t& k, unsigned char* stages, St
         scales[t.blk0] = make_float2(a, q);
     }
     named_sync(kBarCons, kConsumers);
-    const float qm = sh.qm[0], qv = sh.qv[0];
+    const float qm1 = sh.qm[0], qv1 = sh.qv[0];
+    float qm[kV], qv[kV];
+#pragma unroll
+    for (int i = 0; i < kV; ++i) {
+        qm[i] = qm1;
+        qv[i] = qv1;
+    }
     for (int64_t ch = 0; ch < nch; ++ch) {
         if (!wait_stage(sh, k, status)) return false;
         const unsigned char* st = stages + (k % kStages) * kStageBytes;
 #pragma unroll
-        for (int h = 0; h < kHalves; ++h) {
-            const int li = h * (kConsumers * kV) + kV * tid;
+        for (int j = 0; j < kSub; ++j) {
+            const int li = j * (kConsumers * kV) + kV * tid;
             const int64_t vb = a0 + ch * kTile + li;
             if (vb >= hi || vb + kV <= lo) continue;
-            if (vb >= lo && vb + kV <= hi)
-                pass2_one<true>(st, li, vb, lo, hi, dqm, dqv, qm, qv, c, mq, vq);
+            const bool full = vb >= lo && vb + kV <= hi;
+            In4 x;
+            float m[kV], r[kV];
+            if (full)
+                load4<true>(x, st, li, vb, lo, hi, false);
             else
-                pass2_one<false>(st, li, vb, lo, hi, dqm, dqv, qm, qv, c, mq, vq);
+                load4<false>(x, st, li, vb, lo, hi, false);
+#pragma unroll
+            for (int i = 0; i < kV; ++i)
+                new_m_r(g_of(x, i), sbyte_to_f(x.mq, i), ubyte_to_f(x.vq, i), dqm, dqv, c, m[i], r[i]);
+            if (full)
+                store_codes4<true>(m, r, qm, qv, vb, lo, hi, mq, vq);
+            else
+                store_codes4<false>(m, r, qm, qv, vb, lo, hi, mq, vq);
         }
         release_stage(sh, k);
         ++k;
@@ -573,11 +566,11 @@ __device__ bool large_tile(const Tile& t, uint32_t& k, unsigned char* stages, St
 __device__ void zero_tile(const Tile& t, uint16_t* param) {
     const int64_t lo = t.e0, hi = t.e0 + t.n;
     const int64_t a0 = t.e0 & ~int64_t(kAlign - 1);
-    for (int64_t vb = a0 + (int64_t)kV * threadIdx.x; vb < hi; vb += (int64_t)kV * kConsumers) {
-        if (vb >= lo && vb + kV <= hi) {
+    for (int64_t vb = a0 + 8 * (int64_t)threadIdx.x; vb < hi; vb += 8 * (int64_t)kConsumers) {
+        if (vb >= lo && vb + 8 <= hi) {
             __stcs(reinterpret_cast<uint4*>(param + vb), make_uint4(0, 0, 0, 0));
         } else {
-            for (int i = 0; i < kV; ++i)
+            for (int i = 0; i < 8; ++i)
                 if (vb + i >= lo && vb + i < hi) param[vb + i] = 0;
         }
     }
