@@ -56,7 +56,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 void add_zero_tiles(std::vector<Tile>& out, int64_t a, int64_t b) {
     for (int64_t e = a; e < b; e += kZeroChunk)
-        out.push_back(Tile{e, 0, std::min(kZeroChunk, b - e), 0, TILE_ZERO, 0, 0});
+        out.push_back(Tile{e, 0, std::min(kZeroChunk, b - e), 0, TILE_ZERO, 0, 0u});
 }
 
 void build_tiles(const dbuf_plan_s& p, std::vector<Tile>& tiles) {
@@ -73,13 +73,14 @@ void build_tiles(const dbuf_plan_s& p, std::vector<Tile>& tiles) {
                 const int64_t cap = kTile - (e0 & (kAlign - 1));
                 const int64_t q = std::min<int64_t>({kMaxBlk, cap / b, nb - j});
                 if (q >= 1) {
+                    const uint32_t magic = b >= 2 ? (uint32_t)(((uint64_t(1) << 32) + (uint64_t)b - 1) / (uint64_t)b) : 0u;
                     whole.push_back(Tile{e0, blk + j, std::min(q * b, n - j * b), (int32_t)b, TILE_WHOLE,
-                                         (int32_t)q, 0});
+                                         (int32_t)q, magic});
                     j += q;
                     continue;
                 }
             }
-            large.push_back(Tile{e0, blk + j, std::min(b, n - j * b), 0, TILE_LARGE, 1, 0});
+            large.push_back(Tile{e0, blk + j, std::min(b, n - j * b), 0, TILE_LARGE, 1, 0u});
             j += 1;
         }
         blk += nb;

@@ -130,10 +130,9 @@ __device__ __forceinline__ float g_of(const In4& x, int i) {
     return __uint_as_float((i & 1) ? (w & 0xffff0000u) : (w << 16));
 }
 
-// When !FULL only elements in [lo, hi) are taken; the rest read as zero.
+// When !FULL only local elements in [lo, hi) are taken; the rest read as zero.
 template <bool FULL>
-__device__ __forceinline__ void load4(In4& x, const unsigned char* st, int li, int64_t vb, int64_t lo, int64_t hi,
-                                      bool want_p) {
+__device__ __forceinline__ void load4(In4& x, const unsigned char* st, int li, int lo, int hi, bool want_p) {
     if (FULL) {
         const uint2 g = *reinterpret_cast<const uint2*>(st + kOffG + 2 * li);
         x.g[0] = g.x;
@@ -150,13 +149,13 @@ __device__ __forceinline__ void load4(In4& x, const unsigned char* st, int li, i
         uint32_t gw[2] = {0, 0}, a = 0, b = 0;
 #pragma unroll
         for (int i = 0; i < kV; ++i) {
-            const int64_t e = vb + i;
+            const int e = li + i;
             const bool in = (e >= lo && e < hi);
-            x.p[i] = (in && want_p) ? p[li + i] : 0.f;
+            x.p[i] = (in && want_p) ? p[e] : 0.f;
             if (in) {
-                gw[i >> 1] |= (uint32_t)g[li + i] << (16 * (i & 1));
-                a |= (uint32_t)st[kOffMQ + li + i] << (8 * i);
-                b |= (uint32_t)st[kOffVQ + li + i] << (8 * i);
+                gw[i >> 1] |= (uint32_t)g[e] << (16 * (i & 1));
+                a |= (uint32_t)st[kOffMQ + e] << (8 * i);
+                b |= (uint32_t)st[kOffVQ + e] << (8 * i);
             }
         }
         x.g[0] = gw[0];
@@ -183,20 +182,28 @@ __device__ __forceinline__ void unstash_mr(const unsigned char* st, int li, floa
     r[3] = *reinterpret_cast<const float*>(st + kOffVQ + li);
 }
 
+// Global pointers shifted to a window's first element, so the stores take
+// 32-bit local indices.
+struct Out {
+    float* master;
+    uint16_t* param;
+    int8_t* mq;
+    uint8_t* vq;
+};
+
 template <bool FULL>
-__device__ __forceinline__ void store_p4(const float* p, int64_t vb, int64_t lo, int64_t hi, float* master,
-                                         uint16_t* param) {
+__device__ __forceinline__ void store_p4(const float* p, int li, int lo, int hi, const Out& o) {
     const uint2 h = make_uint2(bf16x2_bits(p[0], p[1]), bf16x2_bits(p[2], p[3]));
     if (FULL) {
-        __stcs(reinterpret_cast<float4*>(master + vb), make_float4(p[0], p[1], p[2], p[3]));
-        __stcs(reinterpret_cast<uint2*>(param + vb), h);
+        __stcs(reinterpret_cast<float4*>(o.master + li), make_float4(p[0], p[1], p[2], p[3]));
+        __stcs(reinterpret_cast<uint2*>(o.param + li), h);
     } else {
 #pragma unroll
         for (int i = 0; i < kV; ++i) {
-            const int64_t e = vb + i;
+            const int e = li + i;
             if (e >= lo && e < hi) {
-                master[e] = p[i];
-                param[e] = (uint16_t)(((i < 2) ? h.x : h.y) >> (16 * (i & 1)));
+                o.master[e] = p[i];
+                o.param[e] = (uint16_t)(((i < 2) ? h.x : h.y) >> (16 * (i & 1)));
             }
         }
     }
@@ -205,8 +212,8 @@ __device__ __forceinline__ void store_p4(const float* p, int64_t vb, int64_t lo,
 // Codes of 4 elements.  |m*qm| <= 127 and 0 <= r*qv <= 255 hold by
 // construction (qm = 127/max|m| over the same values), so no clamp is needed.
 template <bool FULL>
-__device__ __forceinline__ void store_codes4(const float* m, const float* r, const float* qm, const float* qv,
-                                             int64_t vb, int64_t lo, int64_t hi, int8_t* mq, uint8_t* vq) {
+__device__ __forceinline__ void store_codes4(const float* m, const float* r, const float* qm, const float* qv, int li,
+                                             int lo, int hi, const Out& o) {
     uint32_t bm[kV], bv[kV];
 #pragma unroll
     for (int i = 0; i < kV; ++i) {
@@ -214,15 +221,15 @@ __device__ __forceinline__ void store_codes4(const float* m, const float* r, con
         bv[i] = rne_low_bits(__fmul_rn(r[i], qv[i]));
     }
     if (FULL) {
-        __stcs(reinterpret_cast<uint32_t*>(mq + vb), pack_low_bytes(bm[0], bm[1], bm[2], bm[3]));
-        __stcs(reinterpret_cast<uint32_t*>(vq + vb), pack_low_bytes(bv[0], bv[1], bv[2], bv[3]));
+        __stcs(reinterpret_cast<uint32_t*>(o.mq + li), pack_low_bytes(bm[0], bm[1], bm[2], bm[3]));
+        __stcs(reinterpret_cast<uint32_t*>(o.vq + li), pack_low_bytes(bv[0], bv[1], bv[2], bv[3]));
     } else {
 #pragma unroll
         for (int i = 0; i < kV; ++i) {
-            const int64_t e = vb + i;
+            const int e = li + i;
             if (e >= lo && e < hi) {
-                mq[e] = (int8_t)(bm[i] & 0xffu);
-                vq[e] = (uint8_t)(bv[i] & 0xffu);
+                o.mq[e] = (int8_t)(bm[i] & 0xffu);
+                o.vq[e] = (uint8_t)(bv[i] & 0xffu);
             }
         }
     }
@@ -230,17 +237,16 @@ __device__ __forceinline__ void store_codes4(const float* m, const float* r, con
 
 // Update of one vector whose elements share dqm/dqv (one block).
 template <bool FULL>
-__device__ __forceinline__ void update4(const unsigned char* st, int li, int64_t vb, int64_t lo, int64_t hi,
-                                        float dqm, float dqv, const StepC& c, float* master, uint16_t* param,
-                                        float* m, float* r) {
+__device__ __forceinline__ void update4(const unsigned char* st, int li, int lo, int hi, float dqm, float dqv,
+                                        const StepC& c, const Out& o, float* m, float* r) {
     In4 x;
-    load4<FULL>(x, st, li, vb, lo, hi, true);
+    load4<FULL>(x, st, li, lo, hi, true);
 #pragma unroll
     for (int i = 0; i < kV; ++i) {
         new_m_r(g_of(x, i), sbyte_to_f(x.mq, i), ubyte_to_f(x.vq, i), dqm, dqv, c, m[i], r[i]);
         x.p[i] = new_p(x.p[i], m[i], r[i], c);
     }
-    store_p4<FULL>(x.p, vb, lo, hi, master, param);
+    store_p4<FULL>(x.p, li, lo, hi, o);
 }
 
 // ------------------------------------------------------------- reductions
@@ -368,14 +374,18 @@ __device__ void step_producer(const Tile* __restrict__ tiles, int64_t n_tiles, i
     }
 }
 
-// Whole blocks: phase 1 updates the weights and stashes m, sqrt(v) in the
+// Kinds of whole-block tiles, fixed per tile.
+enum : int { W_SINGLE = 0, W_MULTI4 = 1, W_MIXED = 2 };
+
+// Whole blocks: phase 1 updates the weights and parks m, sqrt(v) in the
 // stage; block maxima meet in shared memory; phase 2 writes the codes.
-__device__ bool whole_tile(const Tile& t, uint32_t k, unsigned char* stages, StepShared& sh, float* master,
-                           uint16_t* param, int8_t* mq, uint8_t* vq, float2* scales, const StepC& c,
-                           int32_t* status) {
-    if (!wait_stage(sh, k, status)) return false;
+//   W_SINGLE: one block.  W_MULTI4: blocks of a multiple of 4 elements, so
+//   each vector lies in one block, found as umulhi(x, magic) = x / b.
+//   W_MIXED: shorter or odd blocks, per-element block numbers (rare).
+template <int MODE>
+__device__ void whole_tile(const Tile& t, unsigned char* st, StepShared& sh, float* master, uint16_t* param,
+                           int8_t* mq, uint8_t* vq, float2* scales, const StepC& c) {
     const int tid = threadIdx.x;
-    unsigned char* st = stages + (k % kStages) * kStageBytes;
     const int nb = t.nblk;
     if (tid < nb) {
         const float2 sc = reinterpret_cast<const float2*>(st + kOffS)[(t.blk0 & 1) + tid];
@@ -387,57 +397,68 @@ __device__ bool whole_tile(const Tile& t, uint32_t k, unsigned char* stages, Ste
     named_sync(kBarCons, kConsumers);
 
     const int64_t a0 = t.e0 & ~int64_t(kAlign - 1);
-    const int64_t lo = t.e0, hi = t.e0 + t.n;
-    const uint32_t b = (uint32_t)t.b;
-    const bool single = nb == 1;
-    float am1 = 0.f, ar1 = 0.f;  // single block: running max over the thread's vectors
+    const Out o{master + a0, param + a0, mq + a0, vq + a0};
+    const int lo = (int)(t.e0 - a0), hi = lo + (int)t.n;  // local range of the tile's elements
+    const uint32_t b = (uint32_t)t.b, magic = t.magic;
+    float am1 = 0.f, ar1 = 0.f;
 #pragma unroll
     for (int j = 0; j < kSub; ++j) {
         const int li = j * (kConsumers * kV) + kV * tid;
-        const int64_t vb = a0 + li;
-        const int64_t elo = max(vb, lo), ehi = min(vb + kV, hi);
-        const bool any = elo < ehi;
-        const bool full = (vb >= lo) && (vb + kV <= hi);
-        const int bf = any ? (single ? 0 : (int)((uint32_t)(elo - lo) / b)) : -1;
-        const int bl = any ? (single ? 0 : (int)((uint32_t)(ehi - 1 - lo) / b)) : -1;
+        const bool any = li < hi && li + kV > lo;
+        const bool full = li >= lo && li + kV <= hi;
         float m[kV], r[kV];
-        float am = 0.f, ar = 0.f;
-        if (any && bf == bl) {
-            if (full)
-                update4<true>(st, li, vb, lo, hi, sh.dqm[bf], sh.dqv[bf], c, master, param, m, r);
-            else
-                update4<false>(st, li, vb, lo, hi, sh.dqm[bf], sh.dqv[bf], c, master, param, m, r);
+        if (MODE == W_SINGLE) {
+            if (any) {
+                if (full)
+                    update4<true>(st, li, lo, hi, sh.dqm[0], sh.dqv[0], c, o, m, r);
+                else
+                    update4<false>(st, li, lo, hi, sh.dqm[0], sh.dqv[0], c, o, m, r);
 #pragma unroll
-            for (int i = 0; i < kV; ++i) {
-                am = fmaxf(am, fabsf(m[i]));
-                ar = fmaxf(ar, r[i]);
+                for (int i = 0; i < kV; ++i) {
+                    am1 = fmaxf(am1, fabsf(m[i]));
+                    ar1 = fmaxf(ar1, r[i]);
+                }
+                stash_mr(st, li, m, r);
             }
-            stash_mr(st, li, m, r);
-        } else if (any) {
-            // blocks shorter than a vector or off the 4-element grid
-            In4 x;
-            load4<false>(x, st, li, vb, lo, hi, true);
+        } else if (MODE == W_MULTI4) {
+            int key = -1;
+            float am = 0.f, ar = 0.f;
+            if (any) {
+                key = (int)__umulhi((uint32_t)(max(li, lo) - lo), magic);
+                if (full)
+                    update4<true>(st, li, lo, hi, sh.dqm[key], sh.dqv[key], c, o, m, r);
+                else
+                    update4<false>(st, li, lo, hi, sh.dqm[key], sh.dqv[key], c, o, m, r);
 #pragma unroll
-            for (int i = 0; i < kV; ++i) {
-                const int64_t e = vb + i;
-                const int blk = (e < lo || e >= hi) ? bf : (int)((uint32_t)(e - lo) / b);
-                new_m_r(g_of(x, i), sbyte_to_f(x.mq, i), ubyte_to_f(x.vq, i), sh.dqm[blk], sh.dqv[blk], c, m[i],
-                        r[i]);
-                x.p[i] = new_p(x.p[i], m[i], r[i], c);
-                atomicMax(&sh.am[blk], __float_as_uint(fabsf(m[i])));
-                atomicMax(&sh.ar[blk], __float_as_uint(r[i]));
+                for (int i = 0; i < kV; ++i) {
+                    am = fmaxf(am, fabsf(m[i]));
+                    ar = fmaxf(ar, r[i]);
+                }
+                stash_mr(st, li, m, r);
             }
-            store_p4<false>(x.p, vb, lo, hi, master, param);
-            stash_mr(st, li, m, r);
-        }
-        if (single) {
-            am1 = fmaxf(am1, am);
-            ar1 = fmaxf(ar1, ar);
+            block_max_to_smem(key, am, ar, sh);
         } else {
-            block_max_to_smem((any && bf == bl) ? bf : -1, am, ar, sh);
+            if (any) {
+                In4 x;
+                load4<false>(x, st, li, lo, hi, true);
+#pragma unroll
+                for (int i = 0; i < kV; ++i) {
+                    const int e = li + i;
+                    const int blk = (e >= lo && e < hi) ? (int)((uint32_t)(e - lo) / b) : 0;
+                    new_m_r(g_of(x, i), sbyte_to_f(x.mq, i), ubyte_to_f(x.vq, i), sh.dqm[blk], sh.dqv[blk], c, m[i],
+                            r[i]);
+                    x.p[i] = new_p(x.p[i], m[i], r[i], c);
+                    if (e >= lo && e < hi) {
+                        atomicMax(&sh.am[blk], __float_as_uint(fabsf(m[i])));
+                        atomicMax(&sh.ar[blk], __float_as_uint(r[i]));
+                    }
+                }
+                store_p4<false>(x.p, li, lo, hi, o);
+                stash_mr(st, li, m, r);
+            }
         }
     }
-    if (single) block_max_to_smem(0, am1, ar1, sh);
+    if (MODE == W_SINGLE) block_max_to_smem(0, am1, ar1, sh);
     named_sync(kBarCons, kConsumers);
     if (tid < nb) {
         const float AMm = __uint_as_float(sh.am[tid]), AMr = __uint_as_float(sh.ar[tid]);
@@ -449,28 +470,32 @@ __device__ bool whole_tile(const Tile& t, uint32_t k, unsigned char* stages, Ste
 #pragma unroll
     for (int j = 0; j < kSub; ++j) {
         const int li = j * (kConsumers * kV) + kV * tid;
-        const int64_t vb = a0 + li;
-        const int64_t elo = max(vb, lo), ehi = min(vb + kV, hi);
-        if (elo >= ehi) continue;
-        const bool full = (vb >= lo) && (vb + kV <= hi);
+        if (!(li < hi && li + kV > lo)) continue;
+        const bool full = li >= lo && li + kV <= hi;
         float m[kV], r[kV], qm[kV], qv[kV];
         unstash_mr(st, li, m, r);
-        const int bf = single ? 0 : (int)((uint32_t)(elo - lo) / b);
-        const int bl = single ? 0 : (int)((uint32_t)(ehi - 1 - lo) / b);
+        if (MODE == W_MIXED) {
 #pragma unroll
-        for (int i = 0; i < kV; ++i) {
-            const int64_t e = vb + i;
-            const int blk = (bf == bl || e < lo || e >= hi) ? bf : (int)((uint32_t)(e - lo) / b);
-            qm[i] = sh.qm[blk];
-            qv[i] = sh.qv[blk];
+            for (int i = 0; i < kV; ++i) {
+                const int e = li + i;
+                const int blk = (e >= lo && e < hi) ? (int)((uint32_t)(e - lo) / b) : 0;
+                qm[i] = sh.qm[blk];
+                qv[i] = sh.qv[blk];
+            }
+        } else {
+            const int key = MODE == W_SINGLE ? 0 : (int)__umulhi((uint32_t)(max(li, lo) - lo), magic);
+            const float q1 = sh.qm[key], q2 = sh.qv[key];
+#pragma unroll
+            for (int i = 0; i < kV; ++i) {
+                qm[i] = q1;
+                qv[i] = q2;
+            }
         }
         if (full)
-            store_codes4<true>(m, r, qm, qv, vb, lo, hi, mq, vq);
+            store_codes4<true>(m, r, qm, qv, li, lo, hi, o);
         else
-            store_codes4<false>(m, r, qm, qv, vb, lo, hi, mq, vq);
+            store_codes4<false>(m, r, qm, qv, li, lo, hi, o);
     }
-    release_stage(sh, k);
-    return true;
 }
 
 // A block longer than a tile: pass 1 over its chunks updates the weights and
@@ -483,23 +508,24 @@ __device__ bool large_tile(const Tile& t, uint32_t& k, unsigned char* stages, St
     const float2 sc = scales[t.blk0];
     const float dqm = __fdiv_rn(sc.x, 127.f), dqv = __fdiv_rn(sc.y, 255.f);
     const int64_t a0 = t.e0 & ~int64_t(kAlign - 1);
-    const int64_t lo = t.e0, hi = t.e0 + t.n;
     const int64_t nch = large_chunks(t);
 
     float am = 0.f, ar = 0.f;
     for (int64_t ch = 0; ch < nch; ++ch) {
         if (!wait_stage(sh, k, status)) return false;
         const unsigned char* st = stages + (k % kStages) * kStageBytes;
+        const int64_t w0 = a0 + ch * kTile;
+        const Out o{master + w0, param + w0, mq + w0, vq + w0};
+        const int lo = (int)max(t.e0 - w0, (int64_t)0), hi = (int)min(t.e0 + t.n - w0, (int64_t)kTile);
 #pragma unroll
         for (int j = 0; j < kSub; ++j) {
             const int li = j * (kConsumers * kV) + kV * tid;
-            const int64_t vb = a0 + ch * kTile + li;
-            if (vb >= hi || vb + kV <= lo) continue;
+            if (!(li < hi && li + kV > lo)) continue;
             float m[kV], r[kV];
-            if (vb >= lo && vb + kV <= hi)
-                update4<true>(st, li, vb, lo, hi, dqm, dqv, c, master, param, m, r);
+            if (li >= lo && li + kV <= hi)
+                update4<true>(st, li, lo, hi, dqm, dqv, c, o, m, r);
             else
-                update4<false>(st, li, vb, lo, hi, dqm, dqv, c, master, param, m, r);
+                update4<false>(st, li, lo, hi, dqm, dqv, c, o, m, r);
 #pragma unroll
             for (int i = 0; i < kV; ++i) {
                 am = fmaxf(am, fabsf(m[i]));
@@ -537,25 +563,27 @@ __device__ bool large_tile(const Tile& t, uint32_t& k, unsigned char* stages, St
     for (int64_t ch = 0; ch < nch; ++ch) {
         if (!wait_stage(sh, k, status)) return false;
         const unsigned char* st = stages + (k % kStages) * kStageBytes;
+        const int64_t w0 = a0 + ch * kTile;
+        const Out o{master + w0, param + w0, mq + w0, vq + w0};
+        const int lo = (int)max(t.e0 - w0, (int64_t)0), hi = (int)min(t.e0 + t.n - w0, (int64_t)kTile);
 #pragma unroll
         for (int j = 0; j < kSub; ++j) {
             const int li = j * (kConsumers * kV) + kV * tid;
-            const int64_t vb = a0 + ch * kTile + li;
-            if (vb >= hi || vb + kV <= lo) continue;
-            const bool full = vb >= lo && vb + kV <= hi;
+            if (!(li < hi && li + kV > lo)) continue;
+            const bool full = li >= lo && li + kV <= hi;
             In4 x;
             float m[kV], r[kV];
             if (full)
-                load4<true>(x, st, li, vb, lo, hi, false);
+                load4<true>(x, st, li, lo, hi, false);
             else
-                load4<false>(x, st, li, vb, lo, hi, false);
+                load4<false>(x, st, li, lo, hi, false);
 #pragma unroll
             for (int i = 0; i < kV; ++i)
                 new_m_r(g_of(x, i), sbyte_to_f(x.mq, i), ubyte_to_f(x.vq, i), dqm, dqv, c, m[i], r[i]);
             if (full)
-                store_codes4<true>(m, r, qm, qv, vb, lo, hi, mq, vq);
+                store_codes4<true>(m, r, qm, qv, li, lo, hi, o);
             else
-                store_codes4<false>(m, r, qm, qv, vb, lo, hi, mq, vq);
+                store_codes4<false>(m, r, qm, qv, li, lo, hi, o);
         }
         release_stage(sh, k);
         ++k;
@@ -606,7 +634,15 @@ __global__ void __launch_bounds__(kStepThreads, 2)
         if (t.kind == TILE_ZERO) {
             zero_tile(t, param);
         } else if (t.kind == TILE_WHOLE) {
-            if (!whole_tile(t, k, stages, sh, master, param, mq, vq, scales, c, status)) return;
+            if (!wait_stage(sh, k, status)) return;
+            unsigned char* st = stages + (k % kStages) * kStageBytes;
+            if (t.nblk == 1)
+                whole_tile<W_SINGLE>(t, st, sh, master, param, mq, vq, scales, c);
+            else if ((t.b & 3) == 0)
+                whole_tile<W_MULTI4>(t, st, sh, master, param, mq, vq, scales, c);
+            else
+                whole_tile<W_MIXED>(t, st, sh, master, param, mq, vq, scales, c);
+            release_stage(sh, k);
             ++k;
         } else {
             if (!large_tile(t, k, stages, sh, master, param, mq, vq, scales, c, status)) return;

@@ -24,7 +24,7 @@ struct Tile {
     int32_t b;     // block size (WHOLE), 0 otherwise
     int32_t kind;
     int32_t nblk;  // blocks in the entry
-    int32_t pad_;
+    uint32_t magic;  // WHOLE with b >= 2: ceil(2^32 / b), so x / b == umulhi(x, magic) for x < 2^16
 };
 static_assert(sizeof(Tile) == 40, "tile layout");
 

@@ -192,3 +192,12 @@ def test_work_table_covers_bucket_once(name):
         if t["kind"] == 2:
             zmask[t["first_elem"]:t["first_elem"] + t["n_elems"]] = True
     assert np.array_equal(zmask, pad)
+
+
+def test_block_index_reciprocal_is_exact():
+    """Whole-block tiles find a vector's block as umulhi(x, ceil(2^32/b)):
+    exact for every block size 2..4096 and every offset x < 4096 in a tile."""
+    x = np.arange(4096, dtype=np.uint64)
+    for b in range(2, 4097):
+        magic = np.uint64(((1 << 32) + b - 1) // b)
+        assert np.array_equal((x * magic) >> np.uint64(32), x // np.uint64(b)), b
