@@ -11,8 +11,8 @@
 // inputs (bf16 grad, fp32 master, int8/uint8 codes, per-block scales) into a
 // 3-stage shared-memory ring with bulk copies (TMA, cp.async.bulk), so the
 // loads of the next tiles are in flight while the consumers compute and wait
-// at barriers.  Consumers read a stage (16 elements per thread, as four
-// 4-element vectors), write weights and the bf16 copy straight to global
+// at barriers.  Consumers read a stage (16 elements per thread, as two
+// 8-element vectors), write weights and the bf16 copy straight to global
 // memory, put the new m and sqrt(v) back into their own bytes of the stage,
 // reduce each block's absmax, then read m and sqrt(v) back and write the
 // codes.  A LARGE block (longer than a tile) is streamed twice: pass 1
@@ -43,8 +43,8 @@ constexpr int kConsumerWarps = 8;
 constexpr int kConsumers = kConsumerWarps * 32;       // 256 threads
 constexpr int kStepThreads = kConsumers + 32;         // + one producer warp
 constexpr int kStages = 3;
-constexpr int kV = 4;                                 // elements per thread-vector
-constexpr int kSub = kTile / (kConsumers * kV);       // vectors per thread per tile (4)
+constexpr int kV = 8;                                 // elements per thread-vector
+constexpr int kSub = kTile / (kConsumers * kV);       // vectors per thread per tile (2)
 constexpr int kOffG = 0;                              // bf16 grad
 constexpr int kOffP = kOffG + kTile * 2;              // fp32 master
 constexpr int kOffMQ = kOffP + kTile * 4;             // int8 codes of m
@@ -112,41 +112,60 @@ __device__ __forceinline__ float new_p(float p, float m, float r, const StepC& c
 
 // ------------------------------------------------------------ vector I/O
 //
-// Thread-vector = 4 consecutive elements at local index li (a multiple of 4)
-// of a stage.  Its bytes in the stage: grad [2li, 2li+8), master
-// [4li, 4li+16), codes [li, li+4) twice.  After phase 1 the thread's new m
-// goes to its master bytes and its new sqrt(v) to its grad (2 values) and
-// code bytes (1 + 1 values): 16 + 16 bytes that no other thread touches.
+// Thread-vector = 8 consecutive elements at local index li (a multiple of 8)
+// of a stage.  Its bytes in the stage: grad [2li, 2li+16), master
+// [4li, 4li+32), codes [li, li+8) twice.  After phase 1 the thread's new m
+// goes to its master bytes and its new sqrt(v) to its grad (4 values) and
+// code bytes (2 + 2 values): 32 + 32 bytes that no other thread touches.
+// The two 16-byte halves of a thread's master bytes are taken in the order
+// h, 1-h with h = bit 2 of the thread index, so each group of 8 threads
+// covers all 32 banks once per access.
 
-struct In4 {
-    uint32_t g[2];  // bf16 pairs
-    float p[4];
-    uint32_t mq;    // int8 codes, sign bits flipped
-    uint32_t vq;    // uint8 codes
+struct In8 {
+    uint32_t g[4];   // bf16 pairs
+    float p[8];
+    uint32_t mq[2];  // int8 codes, sign bits flipped
+    uint32_t vq[2];  // uint8 codes
 };
 
-__device__ __forceinline__ float g_of(const In4& x, int i) {
+__device__ __forceinline__ float g_of(const In8& x, int i) {
     const uint32_t w = x.g[i >> 1];
     return __uint_as_float((i & 1) ? (w & 0xffff0000u) : (w << 16));
 }
 
+__device__ __forceinline__ int half_order() { return (threadIdx.x >> 2) & 1; }
+
+__device__ __forceinline__ void lds_f8(const unsigned char* base, float* v) {
+    const int h = half_order();
+    const float4 a = *reinterpret_cast<const float4*>(base + 16 * h);
+    const float4 b = *reinterpret_cast<const float4*>(base + 16 * (1 - h));
+    const float4 lo = h ? b : a, hi = h ? a : b;
+    v[0] = lo.x; v[1] = lo.y; v[2] = lo.z; v[3] = lo.w;
+    v[4] = hi.x; v[5] = hi.y; v[6] = hi.z; v[7] = hi.w;
+}
+
+__device__ __forceinline__ void sts_f8(unsigned char* base, const float* v) {
+    const int h = half_order();
+    const float4 lo = make_float4(v[0], v[1], v[2], v[3]), hi = make_float4(v[4], v[5], v[6], v[7]);
+    *reinterpret_cast<float4*>(base + 16 * h) = h ? hi : lo;
+    *reinterpret_cast<float4*>(base + 16 * (1 - h)) = h ? lo : hi;
+}
+
 // When !FULL only local elements in [lo, hi) are taken; the rest read as zero.
 template <bool FULL>
-__device__ __forceinline__ void load4(In4& x, const unsigned char* st, int li, int lo, int hi, bool want_p) {
+__device__ __forceinline__ void load8(In8& x, const unsigned char* st, int li, int lo, int hi, bool want_p) {
     if (FULL) {
-        const uint2 g = *reinterpret_cast<const uint2*>(st + kOffG + 2 * li);
-        x.g[0] = g.x;
-        x.g[1] = g.y;
-        x.mq = *reinterpret_cast<const uint32_t*>(st + kOffMQ + li) ^ 0x80808080u;
-        x.vq = *reinterpret_cast<const uint32_t*>(st + kOffVQ + li);
-        if (want_p) {
-            const float4 p = *reinterpret_cast<const float4*>(st + kOffP + 4 * li);
-            x.p[0] = p.x; x.p[1] = p.y; x.p[2] = p.z; x.p[3] = p.w;
-        }
+        const uint4 g = *reinterpret_cast<const uint4*>(st + kOffG + 2 * li);
+        x.g[0] = g.x; x.g[1] = g.y; x.g[2] = g.z; x.g[3] = g.w;
+        const uint2 a = *reinterpret_cast<const uint2*>(st + kOffMQ + li);
+        const uint2 b = *reinterpret_cast<const uint2*>(st + kOffVQ + li);
+        x.mq[0] = a.x ^ 0x80808080u; x.mq[1] = a.y ^ 0x80808080u;
+        x.vq[0] = b.x; x.vq[1] = b.y;
+        if (want_p) lds_f8(st + kOffP + 4 * li, x.p);
     } else {
         const uint16_t* g = reinterpret_cast<const uint16_t*>(st + kOffG);
         const float* p = reinterpret_cast<const float*>(st + kOffP);
-        uint32_t gw[2] = {0, 0}, a = 0, b = 0;
+        uint32_t gw[4] = {0, 0, 0, 0}, aw[2] = {0, 0}, bw[2] = {0, 0};
 #pragma unroll
         for (int i = 0; i < kV; ++i) {
             const int e = li + i;
@@ -154,32 +173,32 @@ __device__ __forceinline__ void load4(In4& x, const unsigned char* st, int li, i
             x.p[i] = (in && want_p) ? p[e] : 0.f;
             if (in) {
                 gw[i >> 1] |= (uint32_t)g[e] << (16 * (i & 1));
-                a |= (uint32_t)st[kOffMQ + e] << (8 * i);
-                b |= (uint32_t)st[kOffVQ + e] << (8 * i);
+                aw[i >> 2] |= (uint32_t)st[kOffMQ + e] << (8 * (i & 3));
+                bw[i >> 2] |= (uint32_t)st[kOffVQ + e] << (8 * (i & 3));
             }
         }
-        x.g[0] = gw[0];
-        x.g[1] = gw[1];
-        x.mq = a ^ 0x80808080u;
-        x.vq = b;
+        x.g[0] = gw[0]; x.g[1] = gw[1]; x.g[2] = gw[2]; x.g[3] = gw[3];
+        x.mq[0] = aw[0] ^ 0x80808080u; x.mq[1] = aw[1] ^ 0x80808080u;
+        x.vq[0] = bw[0]; x.vq[1] = bw[1];
     }
 }
 
 __device__ __forceinline__ void stash_mr(unsigned char* st, int li, const float* m, const float* r) {
-    *reinterpret_cast<float4*>(st + kOffP + 4 * li) = make_float4(m[0], m[1], m[2], m[3]);
-    *reinterpret_cast<uint2*>(st + kOffG + 2 * li) = make_uint2(__float_as_uint(r[0]), __float_as_uint(r[1]));
-    *reinterpret_cast<float*>(st + kOffMQ + li) = r[2];
-    *reinterpret_cast<float*>(st + kOffVQ + li) = r[3];
+    sts_f8(st + kOffP + 4 * li, m);
+    *reinterpret_cast<uint4*>(st + kOffG + 2 * li) =
+        make_uint4(__float_as_uint(r[0]), __float_as_uint(r[1]), __float_as_uint(r[2]), __float_as_uint(r[3]));
+    *reinterpret_cast<uint2*>(st + kOffMQ + li) = make_uint2(__float_as_uint(r[4]), __float_as_uint(r[5]));
+    *reinterpret_cast<uint2*>(st + kOffVQ + li) = make_uint2(__float_as_uint(r[6]), __float_as_uint(r[7]));
 }
 
 __device__ __forceinline__ void unstash_mr(const unsigned char* st, int li, float* m, float* r) {
-    const float4 a = *reinterpret_cast<const float4*>(st + kOffP + 4 * li);
-    const uint2 b = *reinterpret_cast<const uint2*>(st + kOffG + 2 * li);
-    m[0] = a.x; m[1] = a.y; m[2] = a.z; m[3] = a.w;
-    r[0] = __uint_as_float(b.x);
-    r[1] = __uint_as_float(b.y);
-    r[2] = *reinterpret_cast<const float*>(st + kOffMQ + li);
-    r[3] = *reinterpret_cast<const float*>(st + kOffVQ + li);
+    lds_f8(st + kOffP + 4 * li, m);
+    const uint4 a = *reinterpret_cast<const uint4*>(st + kOffG + 2 * li);
+    const uint2 b = *reinterpret_cast<const uint2*>(st + kOffMQ + li);
+    const uint2 d = *reinterpret_cast<const uint2*>(st + kOffVQ + li);
+    r[0] = __uint_as_float(a.x); r[1] = __uint_as_float(a.y); r[2] = __uint_as_float(a.z); r[3] = __uint_as_float(a.w);
+    r[4] = __uint_as_float(b.x); r[5] = __uint_as_float(b.y);
+    r[6] = __uint_as_float(d.x); r[7] = __uint_as_float(d.y);
 }
 
 // Global pointers shifted to a window's first element, so the stores take
@@ -192,27 +211,30 @@ struct Out {
 };
 
 template <bool FULL>
-__device__ __forceinline__ void store_p4(const float* p, int li, int lo, int hi, const Out& o) {
-    const uint2 h = make_uint2(bf16x2_bits(p[0], p[1]), bf16x2_bits(p[2], p[3]));
+__device__ __forceinline__ void store_p8(const float* p, int li, int lo, int hi, const Out& o) {
+    const uint4 h = make_uint4(bf16x2_bits(p[0], p[1]), bf16x2_bits(p[2], p[3]), bf16x2_bits(p[4], p[5]),
+                               bf16x2_bits(p[6], p[7]));
     if (FULL) {
         __stcs(reinterpret_cast<float4*>(o.master + li), make_float4(p[0], p[1], p[2], p[3]));
-        __stcs(reinterpret_cast<uint2*>(o.param + li), h);
+        __stcs(reinterpret_cast<float4*>(o.master + li) + 1, make_float4(p[4], p[5], p[6], p[7]));
+        __stcs(reinterpret_cast<uint4*>(o.param + li), h);
     } else {
+        const uint32_t hw[4] = {h.x, h.y, h.z, h.w};
 #pragma unroll
         for (int i = 0; i < kV; ++i) {
             const int e = li + i;
             if (e >= lo && e < hi) {
                 o.master[e] = p[i];
-                o.param[e] = (uint16_t)(((i < 2) ? h.x : h.y) >> (16 * (i & 1)));
+                o.param[e] = (uint16_t)(hw[i >> 1] >> (16 * (i & 1)));
             }
         }
     }
 }
 
-// Codes of 4 elements.  |m*qm| <= 127 and 0 <= r*qv <= 255 hold by
+// Codes of 8 elements.  |m*qm| <= 127 and 0 <= r*qv <= 255 hold by
 // construction (qm = 127/max|m| over the same values), so no clamp is needed.
 template <bool FULL>
-__device__ __forceinline__ void store_codes4(const float* m, const float* r, const float* qm, const float* qv, int li,
+__device__ __forceinline__ void store_codes8(const float* m, const float* r, const float* qm, const float* qv, int li,
                                              int lo, int hi, const Out& o) {
     uint32_t bm[kV], bv[kV];
 #pragma unroll
@@ -221,8 +243,10 @@ __device__ __forceinline__ void store_codes4(const float* m, const float* r, con
         bv[i] = rne_low_bits(__fmul_rn(r[i], qv[i]));
     }
     if (FULL) {
-        __stcs(reinterpret_cast<uint32_t*>(o.mq + li), pack_low_bytes(bm[0], bm[1], bm[2], bm[3]));
-        __stcs(reinterpret_cast<uint32_t*>(o.vq + li), pack_low_bytes(bv[0], bv[1], bv[2], bv[3]));
+        __stcs(reinterpret_cast<uint2*>(o.mq + li),
+               make_uint2(pack_low_bytes(bm[0], bm[1], bm[2], bm[3]), pack_low_bytes(bm[4], bm[5], bm[6], bm[7])));
+        __stcs(reinterpret_cast<uint2*>(o.vq + li),
+               make_uint2(pack_low_bytes(bv[0], bv[1], bv[2], bv[3]), pack_low_bytes(bv[4], bv[5], bv[6], bv[7])));
     } else {
 #pragma unroll
         for (int i = 0; i < kV; ++i) {
@@ -237,16 +261,17 @@ __device__ __forceinline__ void store_codes4(const float* m, const float* r, con
 
 // Update of one vector whose elements share dqm/dqv (one block).
 template <bool FULL>
-__device__ __forceinline__ void update4(const unsigned char* st, int li, int lo, int hi, float dqm, float dqv,
+__device__ __forceinline__ void update8(const unsigned char* st, int li, int lo, int hi, float dqm, float dqv,
                                         const StepC& c, const Out& o, float* m, float* r) {
-    In4 x;
-    load4<FULL>(x, st, li, lo, hi, true);
+    In8 x;
+    load8<FULL>(x, st, li, lo, hi, true);
 #pragma unroll
     for (int i = 0; i < kV; ++i) {
-        new_m_r(g_of(x, i), sbyte_to_f(x.mq, i), ubyte_to_f(x.vq, i), dqm, dqv, c, m[i], r[i]);
+        new_m_r(g_of(x, i), sbyte_to_f(x.mq[i >> 2], i & 3), ubyte_to_f(x.vq[i >> 2], i & 3), dqm, dqv, c, m[i],
+                r[i]);
         x.p[i] = new_p(x.p[i], m[i], r[i], c);
     }
-    store_p4<FULL>(x.p, li, lo, hi, o);
+    store_p8<FULL>(x.p, li, lo, hi, o);
 }
 
 // ------------------------------------------------------------- reductions
@@ -375,13 +400,13 @@ __device__ void step_producer(const Tile* __restrict__ tiles, int64_t n_tiles, i
 }
 
 // Kinds of whole-block tiles, fixed per tile.
-enum : int { W_SINGLE = 0, W_MULTI4 = 1, W_MIXED = 2 };
+enum : int { W_SINGLE = 0, W_MULTI8 = 1, W_MIXED = 2 };
 
 // Whole blocks: phase 1 updates the weights and parks m, sqrt(v) in the
 // stage; block maxima meet in shared memory; phase 2 writes the codes.
-//   W_SINGLE: one block.  W_MULTI4: blocks of a multiple of 4 elements, so
+//   W_SINGLE: one block.  W_MULTI8: blocks of a multiple of 8 elements, so
 //   each vector lies in one block, found as umulhi(x, magic) = x / b.
-//   W_MIXED: shorter or odd blocks, per-element block numbers (rare).
+//   W_MIXED: blocks not a multiple of 8 elements, per-element block numbers (rare).
 template <int MODE>
 __device__ void whole_tile(const Tile& t, unsigned char* st, StepShared& sh, float* master, uint16_t* param,
                            int8_t* mq, uint8_t* vq, float2* scales, const StepC& c) {
@@ -410,9 +435,9 @@ __device__ void whole_tile(const Tile& t, unsigned char* st, StepShared& sh, flo
         if (MODE == W_SINGLE) {
             if (any) {
                 if (full)
-                    update4<true>(st, li, lo, hi, sh.dqm[0], sh.dqv[0], c, o, m, r);
+                    update8<true>(st, li, lo, hi, sh.dqm[0], sh.dqv[0], c, o, m, r);
                 else
-                    update4<false>(st, li, lo, hi, sh.dqm[0], sh.dqv[0], c, o, m, r);
+                    update8<false>(st, li, lo, hi, sh.dqm[0], sh.dqv[0], c, o, m, r);
 #pragma unroll
                 for (int i = 0; i < kV; ++i) {
                     am1 = fmaxf(am1, fabsf(m[i]));
@@ -420,15 +445,15 @@ __device__ void whole_tile(const Tile& t, unsigned char* st, StepShared& sh, flo
                 }
                 stash_mr(st, li, m, r);
             }
-        } else if (MODE == W_MULTI4) {
+        } else if (MODE == W_MULTI8) {
             int key = -1;
             float am = 0.f, ar = 0.f;
             if (any) {
                 key = (int)__umulhi((uint32_t)(max(li, lo) - lo), magic);
                 if (full)
-                    update4<true>(st, li, lo, hi, sh.dqm[key], sh.dqv[key], c, o, m, r);
+                    update8<true>(st, li, lo, hi, sh.dqm[key], sh.dqv[key], c, o, m, r);
                 else
-                    update4<false>(st, li, lo, hi, sh.dqm[key], sh.dqv[key], c, o, m, r);
+                    update8<false>(st, li, lo, hi, sh.dqm[key], sh.dqv[key], c, o, m, r);
 #pragma unroll
                 for (int i = 0; i < kV; ++i) {
                     am = fmaxf(am, fabsf(m[i]));
@@ -439,13 +464,13 @@ __device__ void whole_tile(const Tile& t, unsigned char* st, StepShared& sh, flo
             block_max_to_smem(key, am, ar, sh);
         } else {
             if (any) {
-                In4 x;
-                load4<false>(x, st, li, lo, hi, true);
+                In8 x;
+                load8<false>(x, st, li, lo, hi, true);
 #pragma unroll
                 for (int i = 0; i < kV; ++i) {
                     const int e = li + i;
                     const int blk = (e >= lo && e < hi) ? (int)((uint32_t)(e - lo) / b) : 0;
-                    new_m_r(g_of(x, i), sbyte_to_f(x.mq, i), ubyte_to_f(x.vq, i), sh.dqm[blk], sh.dqv[blk], c, m[i],
+                    new_m_r(g_of(x, i), sbyte_to_f(x.mq[i >> 2], i & 3), ubyte_to_f(x.vq[i >> 2], i & 3), sh.dqm[blk], sh.dqv[blk], c, m[i],
                             r[i]);
                     x.p[i] = new_p(x.p[i], m[i], r[i], c);
                     if (e >= lo && e < hi) {
@@ -453,7 +478,7 @@ __device__ void whole_tile(const Tile& t, unsigned char* st, StepShared& sh, flo
                         atomicMax(&sh.ar[blk], __float_as_uint(r[i]));
                     }
                 }
-                store_p4<false>(x.p, li, lo, hi, o);
+                store_p8<false>(x.p, li, lo, hi, o);
                 stash_mr(st, li, m, r);
             }
         }
@@ -492,9 +517,9 @@ __device__ void whole_tile(const Tile& t, unsigned char* st, StepShared& sh, flo
             }
         }
         if (full)
-            store_codes4<true>(m, r, qm, qv, li, lo, hi, o);
+            store_codes8<true>(m, r, qm, qv, li, lo, hi, o);
         else
-            store_codes4<false>(m, r, qm, qv, li, lo, hi, o);
+            store_codes8<false>(m, r, qm, qv, li, lo, hi, o);
     }
 }
 
@@ -523,9 +548,9 @@ __device__ bool large_tile(const Tile& t, uint32_t& k, unsigned char* stages, St
             if (!(li < hi && li + kV > lo)) continue;
             float m[kV], r[kV];
             if (li >= lo && li + kV <= hi)
-                update4<true>(st, li, lo, hi, dqm, dqv, c, o, m, r);
+                update8<true>(st, li, lo, hi, dqm, dqv, c, o, m, r);
             else
-                update4<false>(st, li, lo, hi, dqm, dqv, c, o, m, r);
+                update8<false>(st, li, lo, hi, dqm, dqv, c, o, m, r);
 #pragma unroll
             for (int i = 0; i < kV; ++i) {
                 am = fmaxf(am, fabsf(m[i]));
@@ -571,19 +596,19 @@ __device__ bool large_tile(const Tile& t, uint32_t& k, unsigned char* stages, St
             const int li = j * (kConsumers * kV) + kV * tid;
             if (!(li < hi && li + kV > lo)) continue;
             const bool full = li >= lo && li + kV <= hi;
-            In4 x;
+            In8 x;
             float m[kV], r[kV];
             if (full)
-                load4<true>(x, st, li, lo, hi, false);
+                load8<true>(x, st, li, lo, hi, false);
             else
-                load4<false>(x, st, li, lo, hi, false);
+                load8<false>(x, st, li, lo, hi, false);
 #pragma unroll
             for (int i = 0; i < kV; ++i)
-                new_m_r(g_of(x, i), sbyte_to_f(x.mq, i), ubyte_to_f(x.vq, i), dqm, dqv, c, m[i], r[i]);
+                new_m_r(g_of(x, i), sbyte_to_f(x.mq[i >> 2], i & 3), ubyte_to_f(x.vq[i >> 2], i & 3), dqm, dqv, c, m[i], r[i]);
             if (full)
-                store_codes4<true>(m, r, qm, qv, li, lo, hi, o);
+                store_codes8<true>(m, r, qm, qv, li, lo, hi, o);
             else
-                store_codes4<false>(m, r, qm, qv, li, lo, hi, o);
+                store_codes8<false>(m, r, qm, qv, li, lo, hi, o);
         }
         release_stage(sh, k);
         ++k;
@@ -638,8 +663,8 @@ __global__ void __launch_bounds__(kStepThreads, 2)
             unsigned char* st = stages + (k % kStages) * kStageBytes;
             if (t.nblk == 1)
                 whole_tile<W_SINGLE>(t, st, sh, master, param, mq, vq, scales, c);
-            else if ((t.b & 3) == 0)
-                whole_tile<W_MULTI4>(t, st, sh, master, param, mq, vq, scales, c);
+            else if ((t.b & 7) == 0)
+                whole_tile<W_MULTI8>(t, st, sh, master, param, mq, vq, scales, c);
             else
                 whole_tile<W_MIXED>(t, st, sh, master, param, mq, vq, scales, c);
             release_stage(sh, k);
