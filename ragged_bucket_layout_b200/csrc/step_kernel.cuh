@@ -650,8 +650,13 @@ __global__ void __launch_bounds__(kStepThreads, 2)
         return;
     }
     uint32_t k = 0;
+    // The next table entry is loaded one tile ahead, so its latency hides
+    // behind the current tile.
+    Tile nxt;
+    if ((int64_t)blockIdx.x < n_tiles) nxt = tiles[blockIdx.x];
     for (int64_t ti = blockIdx.x; ti < n_tiles; ti += gridDim.x) {
-        const Tile t = tiles[ti];
+        const Tile t = nxt;
+        if (ti + gridDim.x < n_tiles) nxt = tiles[ti + gridDim.x];
         if (!tile_ok(t, bucket, n_blocks)) {
             if (tid == 0) set_status(status, 2);
             continue;
