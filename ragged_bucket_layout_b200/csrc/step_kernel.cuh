@@ -110,6 +110,48 @@ __device__ __forceinline__ float new_p(float p, float m, float r, const StepC& c
     return __fsub_rn(__fmul_rn(p, c.decay), __fmul_rn(c.step_hat, u));
 }
 
+// The same arithmetic on two elements at once with the paired fp32
+// instructions of sm_100 (__fadd2_rn / __fmul2_rn round each component
+// exactly like __fadd_rn / __fmul_rn, so results are unchanged).
+__device__ __forceinline__ float2 dup(float a) { return make_float2(a, a); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 neg2(float2 a) { return make_float2(-a.x, -a.y); }
+
+// Code bytes i, i+1 of a word as two exact floats (see ubyte_to_f).
+__device__ __forceinline__ float2 ubytes_to_f2(uint32_t w, uint32_t i, float bias) {
+    const float2 x = make_float2(__uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540u | i)),
+                                 __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540u | (i + 1))));
+    return add2(x, dup(-bias));
+}
+
+struct StepC2 {
+    float2 b1, omb1, b2, omb2, eps_hat, step_hat, decay, gscale;
+};
+
+__device__ __forceinline__ StepC2 pairs_of(const StepC& c) {
+    return StepC2{dup(c.b1), dup(c.omb1), dup(c.b2), dup(c.omb2), dup(c.eps_hat), dup(c.step_hat), dup(c.decay),
+                  dup(c.gscale)};
+}
+
+// new_m_r for elements (2j, 2j+1) of a vector.
+__device__ __forceinline__ void new_m_r2(float2 graw, float2 qmf, float2 qvf, float2 dqm, float2 dqv,
+                                         const StepC2& c, float2& m, float2& r) {
+    const float2 g = mul2(graw, c.gscale);
+    const float2 mo = mul2(qmf, dqm);
+    const float2 so = mul2(qvf, dqv);
+    const float2 vo = mul2(so, so);
+    m = add2(mul2(c.b1, mo), mul2(c.omb1, g));
+    const float2 v = add2(mul2(c.b2, vo), mul2(c.omb2, mul2(g, g)));
+    r = make_float2(__fsqrt_rn(v.x), __fsqrt_rn(v.y));
+}
+
+__device__ __forceinline__ float2 new_p2(float2 p, float2 m, float2 r, const StepC2& c) {
+    const float2 d = add2(r, c.eps_hat);
+    const float2 u = make_float2(__fdiv_rn(m.x, d.x), __fdiv_rn(m.y, d.y));
+    return add2(mul2(p, c.decay), neg2(mul2(c.step_hat, u)));
+}
+
 // ------------------------------------------------------------ vector I/O
 //
 // Thread-vector = 8 consecutive elements at local index li (a multiple of 8)
@@ -237,10 +279,15 @@ template <bool FULL>
 __device__ __forceinline__ void store_codes8(const float* m, const float* r, const float* qm, const float* qv, int li,
                                              int lo, int hi, const Out& o) {
     uint32_t bm[kV], bv[kV];
+    const float2 magic = dup(12582912.0f);  // 1.5 * 2^23, see rne_low_bits
 #pragma unroll
-    for (int i = 0; i < kV; ++i) {
-        bm[i] = rne_low_bits(__fmul_rn(m[i], qm[i]));
-        bv[i] = rne_low_bits(__fmul_rn(r[i], qv[i]));
+    for (int j = 0; j < kV / 2; ++j) {
+        const float2 a = add2(mul2(make_float2(m[2 * j], m[2 * j + 1]), make_float2(qm[2 * j], qm[2 * j + 1])), magic);
+        const float2 b = add2(mul2(make_float2(r[2 * j], r[2 * j + 1]), make_float2(qv[2 * j], qv[2 * j + 1])), magic);
+        bm[2 * j] = __float_as_uint(a.x);
+        bm[2 * j + 1] = __float_as_uint(a.y);
+        bv[2 * j] = __float_as_uint(b.x);
+        bv[2 * j + 1] = __float_as_uint(b.y);
     }
     if (FULL) {
         __stcs(reinterpret_cast<uint2*>(o.mq + li),
@@ -259,17 +306,46 @@ __device__ __forceinline__ void store_codes8(const float* m, const float* r, con
     }
 }
 
+// New m and sqrt(v) of a loaded vector whose elements share dqm/dqv.
+__device__ __forceinline__ void mr8(const In8& x, float dqm, float dqv, const StepC2& c, float* m, float* r) {
+    const float2 dqm2 = dup(dqm), dqv2 = dup(dqv);
+#pragma unroll
+    for (int j = 0; j < kV / 2; ++j) {
+        const uint32_t w = x.g[j];
+        const float2 g = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+        const float2 qmf = ubytes_to_f2(x.mq[j >> 1], 2 * (j & 1), 8388736.0f);
+        const float2 qvf = ubytes_to_f2(x.vq[j >> 1], 2 * (j & 1), 8388608.0f);
+        float2 mm, rr;
+        new_m_r2(g, qmf, qvf, dqm2, dqv2, c, mm, rr);
+        m[2 * j] = mm.x;
+        m[2 * j + 1] = mm.y;
+        r[2 * j] = rr.x;
+        r[2 * j + 1] = rr.y;
+    }
+}
+
 // Update of one vector whose elements share dqm/dqv (one block).
 template <bool FULL>
 __device__ __forceinline__ void update8(const unsigned char* st, int li, int lo, int hi, float dqm, float dqv,
-                                        const StepC& c, const Out& o, float* m, float* r) {
+                                        const StepC2& c, const Out& o, float* m, float* r) {
     In8 x;
     load8<FULL>(x, st, li, lo, hi, true);
+    const float2 dqm2 = dup(dqm), dqv2 = dup(dqv);
 #pragma unroll
-    for (int i = 0; i < kV; ++i) {
-        new_m_r(g_of(x, i), sbyte_to_f(x.mq[i >> 2], i & 3), ubyte_to_f(x.vq[i >> 2], i & 3), dqm, dqv, c, m[i],
-                r[i]);
-        x.p[i] = new_p(x.p[i], m[i], r[i], c);
+    for (int j = 0; j < kV / 2; ++j) {
+        const uint32_t w = x.g[j];
+        const float2 g = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+        const float2 qmf = ubytes_to_f2(x.mq[j >> 1], 2 * (j & 1), 8388736.0f);
+        const float2 qvf = ubytes_to_f2(x.vq[j >> 1], 2 * (j & 1), 8388608.0f);
+        float2 mm, rr;
+        new_m_r2(g, qmf, qvf, dqm2, dqv2, c, mm, rr);
+        const float2 pn = new_p2(make_float2(x.p[2 * j], x.p[2 * j + 1]), mm, rr, c);
+        x.p[2 * j] = pn.x;
+        x.p[2 * j + 1] = pn.y;
+        m[2 * j] = mm.x;
+        m[2 * j + 1] = mm.y;
+        r[2 * j] = rr.x;
+        r[2 * j + 1] = rr.y;
     }
     store_p8<FULL>(x.p, li, lo, hi, o);
 }
@@ -424,6 +500,7 @@ __device__ void whole_tile(const Tile& t, unsigned char* st, StepShared& sh, flo
     const int64_t a0 = t.e0 & ~int64_t(kAlign - 1);
     const Out o{master + a0, param + a0, mq + a0, vq + a0};
     const int lo = (int)(t.e0 - a0), hi = lo + (int)t.n;  // local range of the tile's elements
+    const StepC2 c2 = pairs_of(c);
     const uint32_t b = (uint32_t)t.b, magic = t.magic;
     float am1 = 0.f, ar1 = 0.f;
 #pragma unroll
@@ -435,9 +512,9 @@ __device__ void whole_tile(const Tile& t, unsigned char* st, StepShared& sh, flo
         if (MODE == W_SINGLE) {
             if (any) {
                 if (full)
-                    update8<true>(st, li, lo, hi, sh.dqm[0], sh.dqv[0], c, o, m, r);
+                    update8<true>(st, li, lo, hi, sh.dqm[0], sh.dqv[0], c2, o, m, r);
                 else
-                    update8<false>(st, li, lo, hi, sh.dqm[0], sh.dqv[0], c, o, m, r);
+                    update8<false>(st, li, lo, hi, sh.dqm[0], sh.dqv[0], c2, o, m, r);
 #pragma unroll
                 for (int i = 0; i < kV; ++i) {
                     am1 = fmaxf(am1, fabsf(m[i]));
@@ -451,9 +528,9 @@ __device__ void whole_tile(const Tile& t, unsigned char* st, StepShared& sh, flo
             if (any) {
                 key = (int)__umulhi((uint32_t)(max(li, lo) - lo), magic);
                 if (full)
-                    update8<true>(st, li, lo, hi, sh.dqm[key], sh.dqv[key], c, o, m, r);
+                    update8<true>(st, li, lo, hi, sh.dqm[key], sh.dqv[key], c2, o, m, r);
                 else
-                    update8<false>(st, li, lo, hi, sh.dqm[key], sh.dqv[key], c, o, m, r);
+                    update8<false>(st, li, lo, hi, sh.dqm[key], sh.dqv[key], c2, o, m, r);
 #pragma unroll
                 for (int i = 0; i < kV; ++i) {
                     am = fmaxf(am, fabsf(m[i]));
@@ -534,6 +611,7 @@ __device__ bool large_tile(const Tile& t, uint32_t& k, unsigned char* stages, St
     const float dqm = __fdiv_rn(sc.x, 127.f), dqv = __fdiv_rn(sc.y, 255.f);
     const int64_t a0 = t.e0 & ~int64_t(kAlign - 1);
     const int64_t nch = large_chunks(t);
+    const StepC2 c2 = pairs_of(c);
 
     float am = 0.f, ar = 0.f;
     for (int64_t ch = 0; ch < nch; ++ch) {
@@ -548,9 +626,9 @@ __device__ bool large_tile(const Tile& t, uint32_t& k, unsigned char* stages, St
             if (!(li < hi && li + kV > lo)) continue;
             float m[kV], r[kV];
             if (li >= lo && li + kV <= hi)
-                update8<true>(st, li, lo, hi, dqm, dqv, c, o, m, r);
+                update8<true>(st, li, lo, hi, dqm, dqv, c2, o, m, r);
             else
-                update8<false>(st, li, lo, hi, dqm, dqv, c, o, m, r);
+                update8<false>(st, li, lo, hi, dqm, dqv, c2, o, m, r);
 #pragma unroll
             for (int i = 0; i < kV; ++i) {
                 am = fmaxf(am, fabsf(m[i]));
@@ -602,9 +680,7 @@ __device__ bool large_tile(const Tile& t, uint32_t& k, unsigned char* stages, St
                 load8<true>(x, st, li, lo, hi, false);
             else
                 load8<false>(x, st, li, lo, hi, false);
-#pragma unroll
-            for (int i = 0; i < kV; ++i)
-                new_m_r(g_of(x, i), sbyte_to_f(x.mq[i >> 2], i & 3), ubyte_to_f(x.vq[i >> 2], i & 3), dqm, dqv, c, m[i], r[i]);
+            mr8(x, dqm, dqv, c2, m, r);
             if (full)
                 store_codes8<true>(m, r, qm, qv, li, lo, hi, o);
             else
