@@ -111,11 +111,27 @@ __device__ __forceinline__ float new_p(float p, float m, float r, const StepC& c
 }
 
 // The same arithmetic on two elements at once with the paired fp32
-// instructions of sm_100 (__fadd2_rn / __fmul2_rn round each component
-// exactly like __fadd_rn / __fmul_rn, so results are unchanged).
+// instructions of sm_100 (add/mul .f32x2), written as PTX with an explicit
+// .rn rounding modifier: each component is rounded exactly as a scalar
+// add/mul, and a multiply feeding an add is never fused into one FMA (the
+// C++ pair intrinsics were fused under optimisation, which changes results).
 __device__ __forceinline__ float2 dup(float a) { return make_float2(a, a); }
-__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n .reg .b64 ra, rb, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
+        " add.rn.f32x2 rd, ra, rb;\n mov.b64 {%0, %1}, rd;\n}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n .reg .b64 ra, rb, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
+        " mul.rn.f32x2 rd, ra, rb;\n mov.b64 {%0, %1}, rd;\n}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
 __device__ __forceinline__ float2 neg2(float2 a) { return make_float2(-a.x, -a.y); }
 
 // Code bytes i, i+1 of a word as two exact floats (see ubyte_to_f).
