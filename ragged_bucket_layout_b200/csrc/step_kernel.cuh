@@ -111,10 +111,12 @@ __device__ __forceinline__ float new_p(float p, float m, float r, const StepC& c
 }
 
 // The same arithmetic on two elements at once with the paired fp32
-// instructions of sm_100 (add/mul .f32x2), written as PTX with an explicit
-// .rn rounding modifier: each component is rounded exactly as a scalar
-// add/mul, and a multiply feeding an add is never fused into one FMA (the
-// C++ pair intrinsics were fused under optimisation, which changes results).
+// instructions of sm_100 (mul/add .f32x2, written as PTX with .rn): each
+// component is rounded exactly as the scalar instruction.  A paired add
+// whose operands are paired products is fused into one FMA by the
+// assembler (measured: about a third of results move by one ulp), so every
+// add that consumes a product stays scalar (__fadd_rn/__fsub_rn are never
+// fused); only adds of non-products use add2.
 __device__ __forceinline__ float2 dup(float a) { return make_float2(a, a); }
 __device__ __forceinline__ float2 add2(float2 a, float2 b) {
     float2 d;
@@ -132,7 +134,13 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
         : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
     return d;
 }
-__device__ __forceinline__ float2 neg2(float2 a) { return make_float2(-a.x, -a.y); }
+// Scalar sums / differences of two paired products, component by component.
+__device__ __forceinline__ float2 sum_of(float2 a, float2 b) {
+    return make_float2(__fadd_rn(a.x, b.x), __fadd_rn(a.y, b.y));
+}
+__device__ __forceinline__ float2 diff_of(float2 a, float2 b) {
+    return make_float2(__fsub_rn(a.x, b.x), __fsub_rn(a.y, b.y));
+}
 
 // Code bytes i, i+1 of a word as two exact floats (see ubyte_to_f).
 __device__ __forceinline__ float2 ubytes_to_f2(uint32_t w, uint32_t i, float bias) {
@@ -157,15 +165,15 @@ __device__ __forceinline__ void new_m_r2(float2 graw, float2 qmf, float2 qvf, fl
     const float2 mo = mul2(qmf, dqm);
     const float2 so = mul2(qvf, dqv);
     const float2 vo = mul2(so, so);
-    m = add2(mul2(c.b1, mo), mul2(c.omb1, g));
-    const float2 v = add2(mul2(c.b2, vo), mul2(c.omb2, mul2(g, g)));
+    m = sum_of(mul2(c.b1, mo), mul2(c.omb1, g));
+    const float2 v = sum_of(mul2(c.b2, vo), mul2(c.omb2, mul2(g, g)));
     r = make_float2(__fsqrt_rn(v.x), __fsqrt_rn(v.y));
 }
 
 __device__ __forceinline__ float2 new_p2(float2 p, float2 m, float2 r, const StepC2& c) {
-    const float2 d = add2(r, c.eps_hat);
+    const float2 d = sum_of(r, c.eps_hat);  // r ends a square-root sequence: keep the add scalar
     const float2 u = make_float2(__fdiv_rn(m.x, d.x), __fdiv_rn(m.y, d.y));
-    return add2(mul2(p, c.decay), neg2(mul2(c.step_hat, u)));
+    return diff_of(mul2(p, c.decay), mul2(c.step_hat, u));
 }
 
 // ------------------------------------------------------------ vector I/O
@@ -298,8 +306,8 @@ __device__ __forceinline__ void store_codes8(const float* m, const float* r, con
     const float2 magic = dup(12582912.0f);  // 1.5 * 2^23, see rne_low_bits
 #pragma unroll
     for (int j = 0; j < kV / 2; ++j) {
-        const float2 a = add2(mul2(make_float2(m[2 * j], m[2 * j + 1]), make_float2(qm[2 * j], qm[2 * j + 1])), magic);
-        const float2 b = add2(mul2(make_float2(r[2 * j], r[2 * j + 1]), make_float2(qv[2 * j], qv[2 * j + 1])), magic);
+        const float2 a = sum_of(mul2(make_float2(m[2 * j], m[2 * j + 1]), make_float2(qm[2 * j], qm[2 * j + 1])), magic);
+        const float2 b = sum_of(mul2(make_float2(r[2 * j], r[2 * j + 1]), make_float2(qv[2 * j], qv[2 * j + 1])), magic);
         bm[2 * j] = __float_as_uint(a.x);
         bm[2 * j + 1] = __float_as_uint(a.y);
         bv[2 * j] = __float_as_uint(b.x);
