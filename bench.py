@@ -71,7 +71,7 @@ def measured_peak():
 
 def kernel_source_hash():
     h = hashlib.sha256()
-    for f in ("dbuf.cu", "internal.h"):
+    for f in ("dbuf.cu", "internal.h", "step_kernel.cuh", "tma.cuh", "tables.h"):
         h.update(open(os.path.join(ROOT, "ragged_bucket_layout_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -159,6 +159,25 @@ def hp_at(t):
     return dict(synth.HPARAMS, step=t)
 
 
+# ------------------------------------------------------------ ranks
+
+def max_over_ranks(x, dist=None, device="cpu"):
+    """Max of a per-rank float over all ranks (one all-reduce; identity on one rank)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(ms_total_max, steps, world, bytes_per_step):
+    """Whole-job GB/s: every rank moves bytes_per_step per step (weak
+    scaling); time is the slowest rank's."""
+    per_step_ms = ms_total_max / steps
+    return world * bytes_per_step / (per_step_ms * 1e-3) / 1e9, per_step_ms
+
+
 # ------------------------------------------------------------ CPU oracle
 
 def oracle_sample(w, info, offsets, fraction_blocks):
@@ -174,8 +193,7 @@ def oracle_sample(w, info, offsets, fraction_blocks):
     lens = length[sel]
     st = np.concatenate([[0], np.cumsum(lens)[:-1]]).astype(np.int64)
     tot = int(lens.sum())
-    rng = np.random.default_rng(0)
-    arr = dict(p=rng.normal(0, PARAM_SIGMA, tot).astype(np.float32),
+    arr = dict(p=synth.normal_f32(synth.stream_key(w.seed, STREAM_PARAM), 0, tot, PARAM_SIGMA),
                g=synth.normal_bf16(synth.stream_key(w.seed, STREAM_GRAD * 1000 + 1), 0, tot, GRAD_SIGMA),
                mq=np.zeros(tot, np.int8), vq=np.zeros(tot, np.uint8), pb=np.zeros(tot, np.uint16),
                sm=np.zeros(len(sel), np.float32), sv=np.zeros(len(sel), np.float32))
@@ -277,13 +295,6 @@ def run_ours(args):
             dist.barrier()
         torch.cuda.synchronize()
 
-    def max_over_ranks(x):
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     gscale = 1.0 / w.m
     step_no = 0
     for _ in range(args.warmup):
@@ -301,12 +312,11 @@ def run_ours(args):
         ev1.synchronize()
         barrier()
     ms_local = ev0.elapsed_time(ev1)
-    ms = max_over_ranks(ms_local)
+    ms = max_over_ranks(ms_local, dist, "cuda")
     status = D.device_status()
     if status != 0:
         raise RuntimeError(f"device status word {status}")
-    per_step_ms = ms / args.steps
-    value = world * stats["step_bytes"] / (per_step_ms * 1e-3) / 1e9
+    value, per_step_ms = job_throughput(ms, args.steps, world, stats["step_bytes"])
     kernel_gbs = stats["step_bytes"] / (ms_local / args.steps * 1e-3) / 1e9
 
     # ---- end to end through the host-buffer entry point
@@ -327,7 +337,7 @@ def run_ours(args):
         e1.record(stream)
         e1.synchronize()
         barrier()
-        ems = max_over_ranks(e0.elapsed_time(e1)) / args.e2e_steps
+        ems = max_over_ranks(e0.elapsed_time(e1), dist, "cuda") / args.e2e_steps
         e2e = {"value": world * stats["step_bytes"] / (ems * 1e-3) / 1e9, "unit": UNIT,
                "h2d_bytes_per_step": 2 * S, "d2h_bytes_per_step": 2 * S, "ms_per_step": ems,
                "path": "dbuf_adam8_step_host (pinned host grads in, bf16 params out)"}

@@ -1,0 +1,55 @@
+"""Multi-rank host logic of the bench on CPU (gloo, world size 2).
+
+Each rank steps its own bucket (weak scaling, no data-path collective); the
+only collective is the all-reduce that takes the slowest rank's time.  This
+checks that logic with two real processes and the gloo backend.
+"""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        local_ms = [10.0, 25.0][rank]            # rank 1 is the slow one
+        ms = bench.max_over_ranks(local_ms, dist, "cpu")
+        value, per_step = bench.job_throughput(ms, 5, world, 1_000_000_000)
+        dist.barrier()
+        out[rank] = (ms, value, per_step)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_take_the_slowest_time():
+    world = 2
+    port = _free_port()
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.start_processes(_worker, args=(world, port, out), nprocs=world, join=True, start_method="spawn")
+        res = dict(out)
+    for r in range(world):
+        ms, value, per_step = res[r]
+        assert ms == 25.0                        # max over ranks on every rank
+        assert per_step == pytest.approx(5.0)
+        # two ranks x 1 GB per step in 5 ms
+        assert value == pytest.approx(2 * 1e9 / 5e-3 / 1e9)
+
+
+def test_single_rank_is_identity():
+    assert bench.max_over_ranks(3.5) == 3.5
+    v, per = bench.job_throughput(10.0, 10, 1, 2_000_000_000)
+    assert per == 1.0 and v == pytest.approx(2000.0)
