@@ -179,3 +179,86 @@ WORKLOAD_NAMES = tuple(_BUILDERS)
 
 def workload(name):
     return _BUILDERS[name]()
+
+
+# ------------------------------------------------- real-model layer buckets
+#
+# One FSDP bucket per transformer layer, shapes from the public model
+# configurations (recalled; no network to re-check them):
+#   DeepSeek-V3: hidden 7168, MLA (q_lora 1536, kv_lora 512, 128 heads, qk
+#   nope/rope 128/64, v 128), 256 routed experts + 1 shared (intermediate
+#   2048), dense MLP intermediate 18432 in the first 3 layers.
+#   GPT-OSS-120B: hidden 2880, 64 query / 8 KV heads of 64, 128 experts with
+#   fused gate_up 5760x2880 and down 2880x2880 (with biases), sinks.
+# k = rows per quantisation block (1x or 16x row granularity of the pages).
+
+def _k(rows, gran):
+    return min(gran, rows)
+
+
+def deepseek_v3_layer(moe=True, gran=1, m=64):
+    H = 7168
+    t = []
+
+    def mat(name, r, c):
+        t.append(TensorSpec(name, r, c, _k(r, gran)))
+
+    def vec(name, n):
+        t.append(_vec(name, n))
+    vec("input_layernorm", H)
+    mat("q_a_proj", 1536, H)
+    vec("q_a_layernorm", 1536)
+    mat("q_b_proj", 128 * 192, 1536)
+    mat("kv_a_proj_with_mqa", 512 + 64, H)
+    vec("kv_a_layernorm", 512)
+    mat("kv_b_proj", 128 * 256, 512)
+    mat("o_proj", H, 128 * 128)
+    vec("post_attention_layernorm", H)
+    if moe:
+        mat("gate", 256, H)
+        vec("e_score_correction_bias", 256)
+        for e in range(256):
+            mat(f"experts.{e}.gate_proj", 2048, H)
+            mat(f"experts.{e}.up_proj", 2048, H)
+            mat(f"experts.{e}.down_proj", H, 2048)
+        mat("shared.gate_proj", 2048, H)
+        mat("shared.up_proj", 2048, H)
+        mat("shared.down_proj", H, 2048)
+    else:
+        mat("mlp.gate_proj", 18432, H)
+        mat("mlp.up_proj", 18432, H)
+        mat("mlp.down_proj", H, 18432)
+    kind = "moe" if moe else "dense"
+    return Workload(f"deepseek_v3_{kind}_k{gran}_m{m}", t, m=m, seed=6,
+                    description=f"DeepSeek-V3 {kind} layer bucket, {gran}-row blocks")
+
+
+def gpt_oss_120b_layer(gran=1, m=64):
+    H = 2880
+    t = []
+
+    def mat(name, r, c):
+        t.append(TensorSpec(name, r, c, _k(r, gran)))
+
+    def vec(name, n):
+        t.append(_vec(name, n))
+    vec("input_layernorm", H)
+    mat("q_proj", 64 * 64, H)
+    vec("q_proj.bias", 64 * 64)
+    mat("k_proj", 8 * 64, H)
+    vec("k_proj.bias", 8 * 64)
+    mat("v_proj", 8 * 64, H)
+    vec("v_proj.bias", 8 * 64)
+    mat("o_proj", H, 64 * 64)
+    vec("o_proj.bias", H)
+    vec("sinks", 64)
+    vec("post_attention_layernorm", H)
+    mat("router", 128, H)
+    vec("router.bias", 128)
+    for e in range(128):
+        mat(f"experts.{e}.gate_up_proj", 2 * H, H)
+        vec(f"experts.{e}.gate_up_proj.bias", 2 * H)
+        mat(f"experts.{e}.down_proj", H, H)
+        vec(f"experts.{e}.down_proj.bias", H)
+    return Workload(f"gpt_oss_120b_k{gran}_m{m}", t, m=m, seed=7,
+                    description=f"GPT-OSS-120B layer bucket, {gran}-row blocks")
