@@ -56,6 +56,14 @@ def _load():
     lib.orc_step_scalars.argtypes = [f32, f32, f32, f32, f32, i64, P]
     lib.orc_pack.restype = None
     lib.orc_pack.argtypes = [i64, P, P, f32]
+    lib.orc_accumulate.restype = None
+    lib.orc_accumulate.argtypes = [i64, P, P, f32]
+    lib.orc_grad_norm.restype = ctypes.c_double
+    lib.orc_grad_norm.argtypes = [i64, P, f32]
+    lib.orc_clip_coef.restype = ctypes.c_double
+    lib.orc_clip_coef.argtypes = [ctypes.c_double, f32]
+    lib.orc_clipped_scale.restype = ctypes.c_float
+    lib.orc_clipped_scale.argtypes = [ctypes.c_double, f32, f32]
     lib.orc_bf16_round.restype = None
     lib.orc_bf16_round.argtypes = [i64, P, P]
     _lib = lib
@@ -196,6 +204,31 @@ def pack(src_bits, dst_bits, scale):
     assert dst_bits.size >= src_bits.size and dst_bits.flags.c_contiguous
     src = np.ascontiguousarray(src_bits)
     _load().orc_pack(src.size, _ptr(src), _ptr(dst_bits), float(scale))
+
+
+def accumulate(src_bits, dst_bits, scale):
+    """DBuffer group add (gradient accumulation; paper Sec. 5 lists add among
+    the fused group operations): dst = bf16(float(dst) + float(src) * scale)."""
+    assert src_bits.dtype == np.uint16 and dst_bits.dtype == np.uint16
+    assert dst_bits.size >= src_bits.size and dst_bits.flags.c_contiguous
+    src = np.ascontiguousarray(src_bits)
+    _load().orc_accumulate(src.size, _ptr(src), _ptr(dst_bits), float(scale))
+
+
+def grad_norm(g_bits, scale):
+    """L2 norm of float(g) * scale over an array (squares summed in double)."""
+    g = np.ascontiguousarray(g_bits, dtype=np.uint16)
+    return float(_load().orc_grad_norm(g.size, _ptr(g), float(scale)))
+
+
+def clip_coef(norm, max_norm):
+    """Clipping coefficient min(1, max_norm / (norm + 1e-6)) in double."""
+    return float(_load().orc_clip_coef(float(norm), float(max_norm)))
+
+
+def clipped_scale(norm, grad_scale, max_norm):
+    """grad_scale after global-norm clipping, rounded to float once."""
+    return float(_load().orc_clipped_scale(float(norm), float(grad_scale), float(max_norm)))
 
 
 def bf16_round(x):

@@ -390,6 +390,43 @@ void orc_pack(int64_t count, const uint16_t* src, uint16_t* dst, float scale) {
     for (int64_t i = 0; i < count; ++i) dst[i] = bf16_rne(bf16_to_f32(src[i]) * scale);
 }
 
+// DBuffer group "add" (gradient accumulation across micro-batches): one
+// tensor's gradient added into its place in the bucket,
+//   dst[i] = bf16(float(dst[i]) + float(src[i]) * scale).
+void orc_accumulate(int64_t count, const uint16_t* src, uint16_t* dst, float scale) {
+    for (int64_t i = 0; i < count; ++i) {
+        float t = bf16_to_f32(src[i]) * scale;
+        float s = bf16_to_f32(dst[i]) + t;
+        dst[i] = bf16_rne(s);
+    }
+}
+
+// Global L2 norm of the scaled gradient bucket: each element is scaled in
+// fp32 exactly as the step does, squared and summed in double, in order.
+double orc_grad_norm(int64_t count, const uint16_t* g, float scale) {
+    double acc = 0.0;
+    for (int64_t i = 0; i < count; ++i) {
+        double x = (double)(bf16_to_f32(g[i]) * scale);
+        acc += x * x;
+    }
+    return std::sqrt(acc);
+}
+
+// Gradient scale after global-norm clipping (the convention of
+// torch.nn.utils.clip_grad_norm_: coefficient max_norm / (norm + 1e-6),
+// applied only when below 1), folded into the step's grad_scale in double
+// and rounded to float once.
+double orc_clip_coef(double norm, float max_norm) {
+    double coef = (double)max_norm / (norm + 1e-6);
+    return coef < 1.0 ? coef : 1.0;
+}
+
+float orc_clipped_scale(double norm, float grad_scale, float max_norm) {
+    double coef = orc_clip_coef(norm, max_norm);
+    if (coef >= 1.0) return grad_scale;
+    return (float)((double)grad_scale * coef);
+}
+
 // bf16 rounding on its own, for the tests.
 void orc_bf16_round(int64_t count, const float* x, uint16_t* out) {
     for (int64_t i = 0; i < count; ++i) out[i] = bf16_rne(x[i]);

@@ -42,7 +42,13 @@ struct StepC {
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumers = kConsumerWarps * 32;       // 256 threads
 constexpr int kStepThreads = kConsumers + 32;         // + one producer warp
-constexpr int kStages = 3;
+#ifndef DBUF_STEP_STAGES
+#define DBUF_STEP_STAGES 3  // shared-memory ring depth
+#endif
+#ifndef DBUF_STEP_MIN_CTAS
+#define DBUF_STEP_MIN_CTAS 2  // CTAs per SM the register budget is sized for
+#endif
+constexpr int kStages = DBUF_STEP_STAGES;
 constexpr int kV = 8;                                 // elements per thread-vector
 constexpr int kSub = kTile / (kConsumers * kV);       // vectors per thread per tile (2)
 constexpr int kOffG = 0;                              // bf16 grad
@@ -729,7 +735,7 @@ __device__ void zero_tile(const Tile& t, uint16_t* param) {
     }
 }
 
-__global__ void __launch_bounds__(kStepThreads, 2)
+__global__ void __launch_bounds__(kStepThreads, DBUF_STEP_MIN_CTAS)
     adam8_step_kernel(const Tile* __restrict__ tiles, int64_t n_tiles, int64_t bucket, float* master,
                       uint16_t* param, const uint16_t* grad, int8_t* mq, uint8_t* vq, float2* scales,
                       int64_t n_blocks, StepC c, int32_t* status) {
