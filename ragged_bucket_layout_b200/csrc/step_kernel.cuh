@@ -5,11 +5,11 @@
 // so every block is updated and requantised on its own, and the whole
 // bucket goes through one grouped launch instead of one launch per tensor.
 //
-// Persistent kernel, one CTA per slot (two per SM): 8 consumer warps and one
-// producer warp.  The producer walks the CTA's share of the work table
+// Persistent kernel, one CTA per slot (three per SM): 8 consumer warps and
+// one producer warp.  The producer walks the CTA's share of the work table
 // (entries blockIdx.x, blockIdx.x + gridDim.x, ...) and streams each tile's
 // inputs (bf16 grad, fp32 master, int8/uint8 codes, per-block scales) into a
-// 3-stage shared-memory ring with bulk copies (TMA, cp.async.bulk), so the
+// 2-stage shared-memory ring with bulk copies (TMA, cp.async.bulk), so the
 // loads of the next tiles are in flight while the consumers compute and wait
 // at barriers.  Consumers read a stage (16 elements per thread, as two
 // 8-element vectors), write weights and the bf16 copy straight to global
@@ -43,10 +43,10 @@ constexpr int kConsumerWarps = 8;
 constexpr int kConsumers = kConsumerWarps * 32;       // 256 threads
 constexpr int kStepThreads = kConsumers + 32;         // + one producer warp
 #ifndef DBUF_STEP_STAGES
-#define DBUF_STEP_STAGES 3  // shared-memory ring depth
+#define DBUF_STEP_STAGES 2  // shared-memory ring depth
 #endif
 #ifndef DBUF_STEP_MIN_CTAS
-#define DBUF_STEP_MIN_CTAS 2  // CTAs per SM the register budget is sized for
+#define DBUF_STEP_MIN_CTAS 3  // CTAs per SM the register budget is sized for
 #endif
 constexpr int kStages = DBUF_STEP_STAGES;
 constexpr int kV = 8;                                 // elements per thread-vector
