@@ -112,6 +112,14 @@ dbuf_status dbuf_create(const dbuf_plan_t* plan, void* device_base, size_t base_
  * valid until the copy completes on `stream`.  Padding is not touched. */
 dbuf_status dbuf_pack_grads(dbuf_t* db, const void* const* grads_bf16, float scale, void* stream);
 
+/* Gradient accumulation across micro-batches, the DBuffer group "add"
+ * (paper Sec. 5; gist.science "Technische samenvatting" 2C: identical
+ * operations such as add, scale and zero are fused across the tensors of a
+ * bucket): for every tensor i, one launch for the whole bucket,
+ *   grad[offset_i + j] = bf16(float(grad[offset_i + j]) + float(grads_bf16[i][j]) * scale).
+ * Arguments and lifetimes as in dbuf_pack_grads.  Padding is not touched. */
+dbuf_status dbuf_accumulate_grads(dbuf_t* db, const void* const* grads_bf16, float scale, void* stream);
+
 typedef struct {
     float lr, beta1, beta2, eps, weight_decay;
     int64_t step; /* 1-based step number t used in the bias corrections */
@@ -132,6 +140,23 @@ typedef struct {
  * float once.  The bf16 param bucket is set to 0 on every padding element.
  * grad_scale is typically 1/m (the reduce-scatter average). */
 dbuf_status dbuf_adam8_step(dbuf_t* db, const dbuf_adam_hparams* hp, float grad_scale, void* stream);
+
+/* Global L2 norm of the gradient bucket as the step would scale it:
+ * sqrt(sum over the bucket of (float(grad) * grad_scale)^2), each scaled
+ * value rounded to float as in the step, squares summed in double in a
+ * fixed order (deterministic on a given device; padding holds zeros).
+ * Writes the norm (double) to device memory norm_dev on `stream`.  Uses the
+ * bucket's own scratch memory; calls on one bucket must not overlap. */
+dbuf_status dbuf_grad_norm(dbuf_t* db, float grad_scale, double* norm_dev, void* stream);
+
+/* dbuf_adam8_step with global-norm clipping, without a host round trip:
+ * the norm is computed as in dbuf_grad_norm, then the step runs with
+ * grad_scale * min(1, max_norm / (norm + 1e-6)) (formed in double on the
+ * device, rounded to float once; the convention of
+ * torch.nn.utils.clip_grad_norm_).  norm_dev may be NULL; otherwise it
+ * receives the norm.  max_norm > 0. */
+dbuf_status dbuf_adam8_step_clipped(dbuf_t* db, const dbuf_adam_hparams* hp, float grad_scale, float max_norm,
+                                    double* norm_dev, void* stream);
 
 /* The same step with host buffers at both ends (the end-to-end path): copies
  * grads_host (bucket_elems bf16, caller's host memory, pinned for overlap)

@@ -62,6 +62,9 @@ _SIGS = {
     "dbuf_required_bytes": (_sz, [_P]),
     "dbuf_create": (ctypes.c_int, [_P, _P, _sz, _P, _PP]),
     "dbuf_pack_grads": (ctypes.c_int, [_P, _PP, _f32, _P]),
+    "dbuf_accumulate_grads": (ctypes.c_int, [_P, _PP, _f32, _P]),
+    "dbuf_grad_norm": (ctypes.c_int, [_P, _f32, _P, _P]),
+    "dbuf_adam8_step_clipped": (ctypes.c_int, [_P, ctypes.POINTER(dbuf_adam_hparams), _f32, _f32, _P, _P]),
     "dbuf_adam8_step": (ctypes.c_int, [_P, ctypes.POINTER(dbuf_adam_hparams), _f32, _P]),
     "dbuf_adam8_step_host": (ctypes.c_int, [_P, ctypes.POINTER(dbuf_adam_hparams), _f32, _P, _P, _P]),
     "dbuf_unpack_views": (ctypes.c_int, [_P, ctypes.c_int, ctypes.POINTER(dbuf_view)]),
@@ -160,6 +163,21 @@ def _hp(hp):
 def dbuf_pack_grads(db, grad_ptrs, scale, stream=None):
     arr = (ctypes.c_void_p * max(len(grad_ptrs), 1))(*[int(p) for p in grad_ptrs])
     _check(_lib.dbuf_pack_grads(db, arr, float(scale), _stream(stream)))
+
+
+def dbuf_accumulate_grads(db, grad_ptrs, scale, stream=None):
+    arr = (ctypes.c_void_p * max(len(grad_ptrs), 1))(*[int(p) for p in grad_ptrs])
+    _check(_lib.dbuf_accumulate_grads(db, arr, float(scale), _stream(stream)))
+
+
+def dbuf_grad_norm(db, grad_scale, norm_dev_ptr, stream=None):
+    _check(_lib.dbuf_grad_norm(db, float(grad_scale), norm_dev_ptr, _stream(stream)))
+
+
+def dbuf_adam8_step_clipped(db, hp, grad_scale, max_norm, norm_dev_ptr=None, stream=None):
+    h = _hp(hp)
+    _check(_lib.dbuf_adam8_step_clipped(db, ctypes.byref(h), float(grad_scale), float(max_norm), norm_dev_ptr,
+                                        _stream(stream)))
 
 
 def dbuf_adam8_step(db, hp, grad_scale, stream=None):
@@ -278,6 +296,17 @@ class DBuffer:
 
     def pack(self, grads, scale):
         dbuf_pack_grads(self.handle, [g.data_ptr() for g in grads], scale, self.stream)
+
+    def accumulate(self, grads, scale):
+        dbuf_accumulate_grads(self.handle, [g.data_ptr() for g in grads], scale, self.stream)
+
+    def grad_norm(self, grad_scale, out):
+        """Writes the norm into `out` (a float64 CUDA tensor with one element)."""
+        dbuf_grad_norm(self.handle, grad_scale, out.data_ptr(), self.stream)
+
+    def step_clipped(self, hp, grad_scale, max_norm, out=None):
+        dbuf_adam8_step_clipped(self.handle, hp, grad_scale, max_norm, out.data_ptr() if out is not None else None,
+                                self.stream)
 
     def device_status(self):
         return dbuf_get_device_status(self.handle, self.stream)

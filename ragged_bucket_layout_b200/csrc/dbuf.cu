@@ -18,6 +18,7 @@
 #include <string>
 #include <vector>
 
+#include "group_kernels.cuh"
 #include "internal.h"
 #include "pack_kernel.cuh"
 #include "step_kernel.cuh"
@@ -109,7 +110,7 @@ void build_pack_chunks(const dbuf_plan_s& p, std::vector<PackChunk>& chunks, std
 }
 
 struct Layout {
-    size_t master, param, grad, mq, vq, scales, tiles, chunks, status, total;
+    size_t master, param, grad, mq, vq, scales, tiles, chunks, status, scratch, total;
 };
 
 Layout layout_of(const dbuf_plan_s& p, size_t n_tiles, size_t n_chunks) {
@@ -125,6 +126,7 @@ Layout layout_of(const dbuf_plan_s& p, size_t n_tiles, size_t n_chunks) {
     L.tiles = at;  at = align256(at + n_tiles * sizeof(Tile));
     L.chunks = at; at = align256(at + n_chunks * sizeof(PackChunk));
     L.status = at; at = align256(at + 16);
+    L.scratch = at; at = align256(at + sizeof(NormScratch));
     L.total = at;
     return L;
 }
@@ -147,10 +149,12 @@ struct dbuf_s {
     Tile* tiles = nullptr;
     PackChunk* chunks = nullptr;
     int32_t* status = nullptr;
+    NormScratch* scratch = nullptr;
     std::vector<Tile> h_tiles;
     std::vector<PackChunk> h_chunks;
     std::vector<int64_t> h_chunk_first;
     int step_grid = 0;  // persistent CTAs of the step kernel
+    int norm_grid = 1;  // CTAs of the norm reduction
 };
 
 // ----------------------------------------------------------- launches
@@ -256,6 +260,10 @@ extern "C" dbuf_status dbuf_create(const dbuf_plan_t* plan, void* device_base, s
             delete db;
             return gs;
         }
+        int sms = 1;
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, db->device);
+        const int64_t want = (db->plan.bucket / 8 + kNormThreads - 1) / kNormThreads;
+        db->norm_grid = (int)std::max<int64_t>(1, std::min<int64_t>({want, (int64_t)kNormMaxCTAs, 4 * (int64_t)sms}));
     }
     if (device_base) {
         if ((reinterpret_cast<uintptr_t>(device_base) & 255u) != 0 || base_bytes < db->bytes) {
@@ -289,6 +297,7 @@ extern "C" dbuf_status dbuf_create(const dbuf_plan_t* plan, void* device_base, s
     db->tiles = reinterpret_cast<Tile*>(b + db->lay.tiles);
     db->chunks = reinterpret_cast<PackChunk*>(b + db->lay.chunks);
     db->status = reinterpret_cast<int32_t*>(b + db->lay.status);
+    db->scratch = reinterpret_cast<NormScratch*>(b + db->lay.scratch);
     e = cudaMemsetAsync(db->base, 0, db->bytes, st);
     if (e == cudaSuccess && !db->h_tiles.empty())
         e = cudaMemcpyAsync(db->tiles, db->h_tiles.data(), db->h_tiles.size() * sizeof(Tile),
@@ -311,14 +320,15 @@ extern "C" void dbuf_destroy(dbuf_t* db) {
     delete db;
 }
 
-extern "C" dbuf_status dbuf_pack_grads(dbuf_t* db, const void* const* grads_bf16, float scale, void* stream) {
-    if (!db) return fail(DBUF_EINVAL, "dbuf_pack_grads: db is NULL");
-    if (db->plan.n > 0 && !grads_bf16) return fail(DBUF_EINVAL, "dbuf_pack_grads: grads_bf16 is NULL");
+static dbuf_status gather_grads(dbuf_t* db, const void* const* grads_bf16, float scale, void* stream, bool accumulate,
+                                const char* who) {
+    if (!db) return fail(DBUF_EINVAL, std::string(who) + ": db is NULL");
+    if (db->plan.n > 0 && !grads_bf16) return fail(DBUF_EINVAL, std::string(who) + ": grads_bf16 is NULL");
     for (int32_t i = 0; i < db->plan.n; ++i)
         if (!grads_bf16[i] || (reinterpret_cast<uintptr_t>(grads_bf16[i]) & 1u))
-            return fail(DBUF_EINVAL, "dbuf_pack_grads: gradient pointer " + std::to_string(i) +
+            return fail(DBUF_EINVAL, std::string(who) + ": gradient pointer " + std::to_string(i) +
                                          " is NULL or not 2-byte aligned");
-    dbuf_status s = check_device(db, "dbuf_pack_grads");
+    dbuf_status s = check_device(db, who);
     if (s != DBUF_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const size_t smem = kPackChunk * 2;
@@ -329,11 +339,23 @@ extern "C" dbuf_status dbuf_pack_grads(dbuf_t* db, const void* const* grads_bf16
         for (int32_t i = t0; i < t1; ++i) ptrs.p[i - t0] = static_cast<const uint16_t*>(grads_bf16[i]);
         const int64_t c0 = db->h_chunk_first[t0], c1 = db->h_chunk_first[t1];
         if (c1 <= c0) continue;
-        pack_kernel<<<(unsigned)(c1 - c0), kPackThreads, smem, st>>>(ptrs, db->chunks, c0, t0, db->grad,
-                                                                      db->plan.bucket, scale, db->status);
-        CUDA_TRY(cudaGetLastError(), "dbuf_pack_grads: launch");
+        if (accumulate)
+            pack_kernel<true><<<(unsigned)(c1 - c0), kPackThreads, smem, st>>>(ptrs, db->chunks, c0, t0, db->grad,
+                                                                                db->plan.bucket, scale, db->status);
+        else
+            pack_kernel<false><<<(unsigned)(c1 - c0), kPackThreads, smem, st>>>(ptrs, db->chunks, c0, t0, db->grad,
+                                                                                 db->plan.bucket, scale, db->status);
+        CUDA_TRY(cudaGetLastError(), who);
     }
     return DBUF_OK;
+}
+
+extern "C" dbuf_status dbuf_pack_grads(dbuf_t* db, const void* const* grads_bf16, float scale, void* stream) {
+    return gather_grads(db, grads_bf16, scale, stream, false, "dbuf_pack_grads");
+}
+
+extern "C" dbuf_status dbuf_accumulate_grads(dbuf_t* db, const void* const* grads_bf16, float scale, void* stream) {
+    return gather_grads(db, grads_bf16, scale, stream, true, "dbuf_accumulate_grads");
 }
 
 static dbuf_status step_checks(dbuf_t* db, const dbuf_adam_hparams* hp, const char* who) {
@@ -353,8 +375,41 @@ extern "C" dbuf_status dbuf_adam8_step(dbuf_t* db, const dbuf_adam_hparams* hp, 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     adam8_step_kernel<<<(unsigned)db->step_grid, kStepThreads, kStepSmem, st>>>(
         db->tiles, (int64_t)db->h_tiles.size(), db->plan.bucket, db->master, db->param, db->grad, db->mq, db->vq,
-        db->scales, db->plan.n_blocks, c, db->status);
+        db->scales, db->plan.n_blocks, c, nullptr, db->status);
     CUDA_TRY(cudaGetLastError(), "dbuf_adam8_step: launch");
+    return DBUF_OK;
+}
+
+static dbuf_status launch_norm(dbuf_t* db, float grad_scale, float max_norm, int clip, double* norm_dev,
+                               cudaStream_t st, const char* who) {
+    grad_norm_kernel<<<(unsigned)db->norm_grid, kNormThreads, 0, st>>>(db->grad, db->plan.bucket, grad_scale,
+                                                                       max_norm, clip, db->scratch, norm_dev);
+    CUDA_TRY(cudaGetLastError(), std::string(who) + ": norm launch");
+    return DBUF_OK;
+}
+
+extern "C" dbuf_status dbuf_grad_norm(dbuf_t* db, float grad_scale, double* norm_dev, void* stream) {
+    if (!db) return fail(DBUF_EINVAL, "dbuf_grad_norm: db is NULL");
+    if (!norm_dev) return fail(DBUF_EINVAL, "dbuf_grad_norm: norm_dev is NULL");
+    dbuf_status s = check_device(db, "dbuf_grad_norm");
+    if (s != DBUF_OK) return s;
+    return launch_norm(db, grad_scale, 0.f, 0, norm_dev, reinterpret_cast<cudaStream_t>(stream), "dbuf_grad_norm");
+}
+
+extern "C" dbuf_status dbuf_adam8_step_clipped(dbuf_t* db, const dbuf_adam_hparams* hp, float grad_scale,
+                                               float max_norm, double* norm_dev, void* stream) {
+    dbuf_status s = step_checks(db, hp, "dbuf_adam8_step_clipped");
+    if (s != DBUF_OK) return s;
+    if (!(max_norm > 0.f)) return fail(DBUF_EINVAL, "dbuf_adam8_step_clipped: max_norm must be > 0");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    s = launch_norm(db, grad_scale, max_norm, 1, norm_dev, st, "dbuf_adam8_step_clipped");
+    if (s != DBUF_OK) return s;
+    if (db->h_tiles.empty()) return DBUF_OK;
+    const StepC c = make_step_constants(*hp, grad_scale);
+    adam8_step_kernel<<<(unsigned)db->step_grid, kStepThreads, kStepSmem, st>>>(
+        db->tiles, (int64_t)db->h_tiles.size(), db->plan.bucket, db->master, db->param, db->grad, db->mq, db->vq,
+        db->scales, db->plan.n_blocks, c, &db->scratch->gscale_eff, db->status);
+    CUDA_TRY(cudaGetLastError(), "dbuf_adam8_step_clipped: launch");
     return DBUF_OK;
 }
 
@@ -432,5 +487,7 @@ extern "C" dbuf_status dbuf_clear_device_status(dbuf_t* db, void* stream) {
     if (s != DBUF_OK) return s;
     CUDA_TRY(cudaMemsetAsync(db->status, 0, sizeof(int32_t), reinterpret_cast<cudaStream_t>(stream)),
              "dbuf_clear_device_status");
+    CUDA_TRY(cudaMemsetAsync(&db->scratch->counter, 0, sizeof(uint32_t), reinterpret_cast<cudaStream_t>(stream)),
+             "dbuf_clear_device_status: norm counter");
     return DBUF_OK;
 }

@@ -26,6 +26,15 @@ __device__ __forceinline__ uint16_t scaled_bf16(uint32_t h, float scale) {
     return __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(bf16_bits_to_f32(h), scale)));
 }
 
+__device__ __forceinline__ uint16_t accumulated_bf16(uint32_t d, uint32_t h, float scale) {
+    const float t = __fmul_rn(bf16_bits_to_f32(h), scale);
+    return __bfloat16_as_ushort(__float2bfloat16_rn(__fadd_rn(bf16_bits_to_f32(d), t)));
+}
+
+// ACCUM = false: grad[dst] = bf16(float(src) * scale)           (copy-in)
+// ACCUM = true:  grad[dst] = bf16(float(grad[dst]) + float(src) * scale)
+//                (gradient accumulation, the DBuffer group add)
+template <bool ACCUM>
 __global__ void __launch_bounds__(kPackThreads) pack_kernel(PackPtrs ptrs, const PackChunk* __restrict__ chunks,
                                                             int64_t first_chunk, int32_t tensor_base,
                                                             uint16_t* grad, int64_t bucket, float scale,
@@ -53,7 +62,8 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(PackPtrs ptrs, const
         if (nbulk > 0) bulk_g2s(sbuf, src, (uint32_t)nbulk * 2u, &bar);
     }
     // Element-wise tail while the bulk copy is in flight.
-    for (int32_t i = nbulk + threadIdx.x; i < ch.count; i += kPackThreads) dst[i] = scaled_bf16(src[i], scale);
+    for (int32_t i = nbulk + threadIdx.x; i < ch.count; i += kPackThreads)
+        dst[i] = ACCUM ? accumulated_bf16(dst[i], src[i], scale) : scaled_bf16(src[i], scale);
     if (!mbar_wait_bounded(&bar, 0)) {
         if (threadIdx.x == 0) set_status(status, 1);
         mbar_wait_bounded(&bar, 0);  // let the copy land before the CTA goes away
@@ -63,9 +73,19 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(PackPtrs ptrs, const
         const uint4 w = sbuf[v];
         const uint32_t in[4] = {w.x, w.y, w.z, w.w};
         uint32_t out[4];
+        if (ACCUM) {
+            const uint4 dv = *(reinterpret_cast<const uint4*>(dst) + v);
+            const uint32_t dw[4] = {dv.x, dv.y, dv.z, dv.w};
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-            out[q] = (uint32_t)scaled_bf16(in[q] & 0xffffu, scale) | ((uint32_t)scaled_bf16(in[q] >> 16, scale) << 16);
+            for (int q = 0; q < 4; ++q)
+                out[q] = (uint32_t)accumulated_bf16(dw[q] & 0xffffu, in[q] & 0xffffu, scale) |
+                         ((uint32_t)accumulated_bf16(dw[q] >> 16, in[q] >> 16, scale) << 16);
+        } else {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                out[q] = (uint32_t)scaled_bf16(in[q] & 0xffffu, scale) |
+                         ((uint32_t)scaled_bf16(in[q] >> 16, scale) << 16);
+        }
         __stcs(reinterpret_cast<uint4*>(dst) + v, make_uint4(out[0], out[1], out[2], out[3]));
     }
 }

@@ -738,10 +738,14 @@ __device__ void zero_tile(const Tile& t, uint16_t* param) {
 __global__ void __launch_bounds__(kStepThreads, DBUF_STEP_MIN_CTAS)
     adam8_step_kernel(const Tile* __restrict__ tiles, int64_t n_tiles, int64_t bucket, float* master,
                       uint16_t* param, const uint16_t* grad, int8_t* mq, uint8_t* vq, float2* scales,
-                      int64_t n_blocks, StepC c, int32_t* status) {
+                      int64_t n_blocks, StepC cp, const float* gscale_dev, int32_t* status) {
     extern __shared__ __align__(128) unsigned char stages[];
     __shared__ StepShared sh;
     const int tid = threadIdx.x;
+    // grad_scale comes from device memory when a preceding kernel chose it
+    // (global-norm clipping), so no host round trip is needed.
+    StepC c = cp;
+    if (gscale_dev) c.gscale = *gscale_dev;
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sh.full[s], 1);
