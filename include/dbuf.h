@@ -149,6 +149,26 @@ dbuf_status dbuf_adam8_step(dbuf_t* db, const dbuf_adam_hparams* hp, float grad_
  * bucket's own scratch memory; calls on one bucket must not overlap. */
 dbuf_status dbuf_grad_norm(dbuf_t* db, float grad_scale, double* norm_dev, void* stream);
 
+/* The gradient norm of dbuf_grad_norm for callers that cannot allocate
+ * device memory: code running where cudaMalloc is not allowed or not wanted
+ * (inside a custom allocator or memory-pool callback, a runtime that owns
+ * every byte of device memory, a latency-critical loop that must not touch
+ * the allocator).  It needs no dbuf: grad_bf16 (device, 16-byte aligned) and
+ * n_elems are the input, norm_dev (device, one double) the output:
+ *   sqrt(sum over i < n_elems of (float(grad_bf16[i]) * grad_scale)^2).
+ * No counterpart in the paper: an addition for such callers.
+ * It allocates nothing.  Its scratch (one partial sum per 2^20 elements,
+ * 2048 sums) is a file-scope device array of the library that every GPU
+ * loading the library holds until the process exits; so n_elems is at most
+ * 2^31 and larger sizes return DBUF_EINVAL.  The first call on each device
+ * looks up the array's device address (cudaGetSymbolAddress): make that
+ * first call before any stream capture.  Every call shares the one array,
+ * so calls whose work overlaps on the GPU race and give wrong results;
+ * serialise them (one stream, or events).  Summation order differs from
+ * dbuf_grad_norm's, so results agree to fp64 rounding, not bit for bit. */
+dbuf_status dbuf_grad_norm_noalloc(const void* grad_bf16, int64_t n_elems, float grad_scale, double* norm_dev,
+                                   void* stream);
+
 /* dbuf_adam8_step with global-norm clipping, without a host round trip:
  * the norm is computed as in dbuf_grad_norm, then the step runs with
  * grad_scale * min(1, max_norm / (norm + 1e-6)) (formed in double on the

@@ -64,6 +64,7 @@ _SIGS = {
     "dbuf_pack_grads": (ctypes.c_int, [_P, _PP, _f32, _P]),
     "dbuf_accumulate_grads": (ctypes.c_int, [_P, _PP, _f32, _P]),
     "dbuf_grad_norm": (ctypes.c_int, [_P, _f32, _P, _P]),
+    "dbuf_grad_norm_noalloc": (ctypes.c_int, [_P, _i64, _f32, _P, _P]),
     "dbuf_adam8_step_clipped": (ctypes.c_int, [_P, ctypes.POINTER(dbuf_adam_hparams), _f32, _f32, _P, _P]),
     "dbuf_adam8_step": (ctypes.c_int, [_P, ctypes.POINTER(dbuf_adam_hparams), _f32, _P]),
     "dbuf_adam8_step_host": (ctypes.c_int, [_P, ctypes.POINTER(dbuf_adam_hparams), _f32, _P, _P, _P]),
@@ -172,6 +173,11 @@ def dbuf_accumulate_grads(db, grad_ptrs, scale, stream=None):
 
 def dbuf_grad_norm(db, grad_scale, norm_dev_ptr, stream=None):
     _check(_lib.dbuf_grad_norm(db, float(grad_scale), norm_dev_ptr, _stream(stream)))
+
+
+def dbuf_grad_norm_noalloc(grad_ptr, n_elems, grad_scale, norm_dev_ptr, stream=None):
+    """Allocation-free gradient norm over a plain bf16 device array."""
+    _check(_lib.dbuf_grad_norm_noalloc(grad_ptr, int(n_elems), float(grad_scale), norm_dev_ptr, _stream(stream)))
 
 
 def dbuf_adam8_step_clipped(db, hp, grad_scale, max_norm, norm_dev_ptr=None, stream=None):

@@ -14,6 +14,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <string>
 #include <vector>
@@ -394,6 +395,61 @@ extern "C" dbuf_status dbuf_grad_norm(dbuf_t* db, float grad_scale, double* norm
     dbuf_status s = check_device(db, "dbuf_grad_norm");
     if (s != DBUF_OK) return s;
     return launch_norm(db, grad_scale, 0.f, 0, norm_dev, reinterpret_cast<cudaStream_t>(stream), "dbuf_grad_norm");
+}
+
+// ------------------------------------------------ allocation-free norm
+//
+// For callers that cannot allocate device memory: code running where
+// cudaMalloc is not allowed or not wanted (inside a custom allocator or a
+// memory-pool callback, a runtime that owns every byte of device memory, a
+// latency-critical loop that must not hit the allocator).  The norm
+// reduction's scratch lives in this file-scope array instead: every GPU that
+// loads the library holds it until the process exits.  One partial sum per
+// CTA, one CTA per 2^20 elements, so one call covers at most 2^31 elements.
+
+constexpr int64_t kNoAllocChunk = int64_t(1) << 20;
+constexpr int64_t kNoAllocMaxElems = kNoAllocChunk * kNormMaxCTAs;  // 2^31
+
+static __device__ __align__(256) NormScratch g_noalloc_norm_scratch;
+
+namespace {
+std::mutex g_noalloc_mu;
+NormScratch* g_noalloc_ptr[256] = {nullptr};  // device address of the array, per device
+}  // namespace
+
+extern "C" dbuf_status dbuf_grad_norm_noalloc(const void* grad_bf16, int64_t n_elems, float grad_scale,
+                                              double* norm_dev, void* stream) {
+    const char* who = "dbuf_grad_norm_noalloc";
+    if (n_elems < 0 || n_elems > kNoAllocMaxElems)
+        return fail(DBUF_EINVAL, std::string(who) + ": n_elems must be in [0, 2^31] (the static scratch holds " +
+                                     std::to_string(kNormMaxCTAs) + " partial sums of 2^20 elements each)");
+    if (!norm_dev) return fail(DBUF_EINVAL, std::string(who) + ": norm_dev is NULL");
+    if (n_elems > 0 && (!grad_bf16 || (reinterpret_cast<uintptr_t>(grad_bf16) & 15u)))
+        return fail(DBUF_EINVAL, std::string(who) + ": grad_bf16 must be a 16-byte aligned device pointer");
+    int dev = -1;
+    CUDA_TRY(cudaGetDevice(&dev), who);
+    if (dev < 0 || dev >= 256) return fail(DBUF_EINVAL, std::string(who) + ": device ordinal out of range");
+    NormScratch* sc = nullptr;
+    {
+        // First call on a device: find the array's device address (host code
+        // only holds a stand-in for it).
+        std::lock_guard<std::mutex> lock(g_noalloc_mu);
+        if (!g_noalloc_ptr[dev]) {
+            void* p = nullptr;
+            CUDA_TRY(cudaGetSymbolAddress(&p, g_noalloc_norm_scratch), std::string(who) + ": scratch address");
+            g_noalloc_ptr[dev] = static_cast<NormScratch*>(p);
+        }
+        sc = g_noalloc_ptr[dev];
+    }
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // The array keeps the last call's contents; the completion counter must
+    // start at zero (a call that stopped early could have left it set).
+    CUDA_TRY(cudaMemsetAsync(&sc->counter, 0, sizeof(uint32_t), st), std::string(who) + ": reset counter");
+    const int grid = (int)std::max<int64_t>(1, (n_elems + kNoAllocChunk - 1) / kNoAllocChunk);
+    grad_norm_kernel<<<(unsigned)grid, kNormThreads, 0, st>>>(static_cast<const uint16_t*>(grad_bf16), n_elems,
+                                                              grad_scale, 0.f, 0, sc, norm_dev);
+    CUDA_TRY(cudaGetLastError(), std::string(who) + ": launch");
+    return DBUF_OK;
 }
 
 extern "C" dbuf_status dbuf_adam8_step_clipped(dbuf_t* db, const dbuf_adam_hparams* hp, float grad_scale,
