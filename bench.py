@@ -369,6 +369,30 @@ def run_ours(args):
                    "copy_in_path_ms": path_ms, "zero_copy_path_ms": ms_local / args.steps,
                    "copy_bytes": stats["copy_in_bytes"], "tensors": len(sep),
                    "saved_ms": path_ms - ms_local / args.steps}
+        # DBuffer group operations beyond scale/zero on the same bucket:
+        # accumulate (6 B/param), norm (2 B/bucket element), clipped step.
+        norm_out = torch.zeros(1, dtype=torch.float64, device="cuda")
+        with torch.cuda.stream(stream):
+            b0, b1, b2, b3 = (torch.cuda.Event(enable_timing=True) for _ in range(4))
+            D.accumulate(sep, gscale)
+            D.grad_norm(gscale, norm_out)
+            b0.record(stream)
+            for _ in range(reps):
+                D.accumulate(sep, gscale)
+            b1.record(stream)
+            for _ in range(reps):
+                D.grad_norm(gscale, norm_out)
+            b2.record(stream)
+            for _ in range(reps):
+                step_no += 1
+                D.step_clipped(hp_at(step_no), gscale, 1.0, norm_out)
+            b3.record(stream)
+        b3.synchronize()
+        acc_ms, norm_ms, clip_ms = b0.elapsed_time(b1) / reps, b1.elapsed_time(b2) / reps, b2.elapsed_time(b3) / reps
+        copy_in["group_ops"] = {
+            "accumulate_gbs": 6 * stats["params"] / (acc_ms * 1e-3) / 1e9, "accumulate_ms": acc_ms,
+            "grad_norm_gbs": 2 * stats["bucket"] / (norm_ms * 1e-3) / 1e9, "grad_norm_ms": norm_ms,
+            "clipped_step_ms": clip_ms, "clipped_step_gbs": (stats["step_bytes"] + 2 * stats["bucket"]) / (clip_ms * 1e-3) / 1e9}
         del sep
 
     peak, peak_src = measured_peak()
