@@ -27,6 +27,7 @@
 
 #include <cuda_bf16.h>
 
+#include "fastmath.cuh"
 #include "tables.h"
 #include "tma.cuh"
 
@@ -164,16 +165,30 @@ __device__ __forceinline__ StepC2 pairs_of(const StepC& c) {
                   dup(c.gscale)};
 }
 
-// new_m_r for elements (2j, 2j+1) of a vector.
-__device__ __forceinline__ void new_m_r2(float2 graw, float2 qmf, float2 qvf, float2 dqm, float2 dqv,
-                                         const StepC2& c, float2& m, float2& r) {
+// New m and v for elements (2j, 2j+1) of a vector (sqrt(v) taken per vector).
+__device__ __forceinline__ void new_m_v2(float2 graw, float2 qmf, float2 qvf, float2 dqm, float2 dqv,
+                                         const StepC2& c, float2& m, float2& v) {
     const float2 g = mul2(graw, c.gscale);
     const float2 mo = mul2(qmf, dqm);
     const float2 so = mul2(qvf, dqv);
     const float2 vo = mul2(so, so);
     m = sum_of(mul2(c.b1, mo), mul2(c.omb1, g));
-    const float2 v = sum_of(mul2(c.b2, vo), mul2(c.omb2, mul2(g, g)));
-    r = make_float2(__fsqrt_rn(v.x), __fsqrt_rn(v.y));
+    v = sum_of(mul2(c.b2, vo), mul2(c.omb2, mul2(g, g)));
+}
+
+// Correctly rounded sqrt of the 4 pairs of a vector: the fast sequence
+// when every v is in its checked range (the normal case), else IEEE sqrt.
+__device__ __forceinline__ void sqrt_vec(const float2* v, float2* r) {
+    uint32_t lo = 0xffffffffu;
+#pragma unroll
+    for (int j = 0; j < kV / 2; ++j) lo = min(lo, min(__float_as_uint(v[j].x), __float_as_uint(v[j].y)));
+    if (lo >= kSqrtFastMinBits) {
+#pragma unroll
+        for (int j = 0; j < kV / 2; ++j) r[j] = sqrt2_fast(v[j]);
+    } else {
+#pragma unroll
+        for (int j = 0; j < kV / 2; ++j) r[j] = make_float2(__fsqrt_rn(v[j].x), __fsqrt_rn(v[j].y));
+    }
 }
 
 __device__ __forceinline__ float2 new_p2(float2 p, float2 m, float2 r, const StepC2& c) {
@@ -339,18 +354,22 @@ __device__ __forceinline__ void store_codes8(const float* m, const float* r, con
 // New m and sqrt(v) of a loaded vector whose elements share dqm/dqv.
 __device__ __forceinline__ void mr8(const In8& x, float dqm, float dqv, const StepC2& c, float* m, float* r) {
     const float2 dqm2 = dup(dqm), dqv2 = dup(dqv);
+    float2 mm[kV / 2], vv[kV / 2], rr[kV / 2];
 #pragma unroll
     for (int j = 0; j < kV / 2; ++j) {
         const uint32_t w = x.g[j];
         const float2 g = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
         const float2 qmf = ubytes_to_f2(x.mq[j >> 1], 2 * (j & 1), 8388736.0f);
         const float2 qvf = ubytes_to_f2(x.vq[j >> 1], 2 * (j & 1), 8388608.0f);
-        float2 mm, rr;
-        new_m_r2(g, qmf, qvf, dqm2, dqv2, c, mm, rr);
-        m[2 * j] = mm.x;
-        m[2 * j + 1] = mm.y;
-        r[2 * j] = rr.x;
-        r[2 * j + 1] = rr.y;
+        new_m_v2(g, qmf, qvf, dqm2, dqv2, c, mm[j], vv[j]);
+    }
+    sqrt_vec(vv, rr);
+#pragma unroll
+    for (int j = 0; j < kV / 2; ++j) {
+        m[2 * j] = mm[j].x;
+        m[2 * j + 1] = mm[j].y;
+        r[2 * j] = rr[j].x;
+        r[2 * j + 1] = rr[j].y;
     }
 }
 
@@ -360,22 +379,13 @@ __device__ __forceinline__ void update8(const unsigned char* st, int li, int lo,
                                         const StepC2& c, const Out& o, float* m, float* r) {
     In8 x;
     load8<FULL>(x, st, li, lo, hi, true);
-    const float2 dqm2 = dup(dqm), dqv2 = dup(dqv);
+    mr8(x, dqm, dqv, c, m, r);
 #pragma unroll
     for (int j = 0; j < kV / 2; ++j) {
-        const uint32_t w = x.g[j];
-        const float2 g = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
-        const float2 qmf = ubytes_to_f2(x.mq[j >> 1], 2 * (j & 1), 8388736.0f);
-        const float2 qvf = ubytes_to_f2(x.vq[j >> 1], 2 * (j & 1), 8388608.0f);
-        float2 mm, rr;
-        new_m_r2(g, qmf, qvf, dqm2, dqv2, c, mm, rr);
-        const float2 pn = new_p2(make_float2(x.p[2 * j], x.p[2 * j + 1]), mm, rr, c);
+        const float2 pn = new_p2(make_float2(x.p[2 * j], x.p[2 * j + 1]), make_float2(m[2 * j], m[2 * j + 1]),
+                                 make_float2(r[2 * j], r[2 * j + 1]), c);
         x.p[2 * j] = pn.x;
         x.p[2 * j + 1] = pn.y;
-        m[2 * j] = mm.x;
-        m[2 * j + 1] = mm.y;
-        r[2 * j] = rr.x;
-        r[2 * j + 1] = rr.y;
     }
     store_p8<FULL>(x.p, li, lo, hi, o);
 }
