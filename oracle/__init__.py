@@ -231,6 +231,68 @@ def clipped_scale(norm, grad_scale, max_norm):
     return float(_load().orc_clipped_scale(float(norm), float(grad_scale), float(max_norm)))
 
 
+def rowwise_layout(rows, cols, m):
+    """Row-wise even sharding, the FSDP2 / Megatron-FSDP baseline of the
+    veScale-FSDP pages (comparison of sharding formats, "row-wise" entry):
+    tensor t is cut along dim 0 into m shards of q_t = ceil(rows_t / m) rows
+    (the last shards shorter or empty) and each shard is padded to q_t rows in
+    the communication buffer.  Rank r's chunk concatenates its padded shards
+    of every tensor in order; an AllGather output holds the m chunks in rank
+    order.  Returns (q, offsets of each tensor's shard within a chunk, chunk
+    size in elements)."""
+    rows = np.asarray(rows, dtype=np.int64)
+    cols = np.asarray(cols, dtype=np.int64)
+    q = (rows + m - 1) // m
+    sizes = q * cols
+    off = np.concatenate([[0], np.cumsum(sizes)[:-1]]).astype(np.int64)
+    return q, off, int(sizes.sum())
+
+
+def _rowwise_rows(rows_t, q_t, r):
+    r0 = r * q_t
+    return r0, max(r0, min(rows_t, r0 + q_t))
+
+
+def rowwise_copy_out(gathered_bits, rows, cols, m):
+    """Interleaved copy-out after the AllGather of the row-wise baseline (the
+    pages' per-parameter copy-out with interleaved addresses): tensor t's rows
+    [r q_t, min(rows_t, (r+1) q_t)) are the first rows of its shard in chunk r.
+    Returns one bf16-bits array of rows_t * cols_t elements per tensor."""
+    q, off, C = rowwise_layout(rows, cols, m)
+    outs = []
+    for t in range(len(q)):
+        n_t = int(rows[t]) * int(cols[t])
+        out = np.zeros(n_t, dtype=np.uint16)
+        for r in range(m):
+            r0, r1 = _rowwise_rows(int(rows[t]), int(q[t]), r)
+            k = (r1 - r0) * int(cols[t])
+            src = r * C + int(off[t])
+            out[r0 * int(cols[t]):r0 * int(cols[t]) + k] = gathered_bits[src:src + k]
+        outs.append(out)
+    return outs
+
+
+def rowwise_copy_in(grads_bits, rows, cols, m, scale):
+    """Interleaved copy-in before the ReduceScatter of the row-wise baseline
+    (the pages' per-parameter copy-in): each tensor's rows go to the shard of
+    the rank that owns them as bf16(float(g) * scale); padding rows are zero.
+    Returns the m * chunk bf16-bits buffer."""
+    q, off, C = rowwise_layout(rows, cols, m)
+    buf = np.zeros(m * C, dtype=np.uint16)
+    for t in range(len(q)):
+        g = np.ascontiguousarray(grads_bits[t], dtype=np.uint16).reshape(-1)
+        for r in range(m):
+            r0, r1 = _rowwise_rows(int(rows[t]), int(q[t]), r)
+            k = (r1 - r0) * int(cols[t])
+            if k == 0:
+                continue
+            dst = r * C + int(off[t])
+            seg = np.zeros(k, dtype=np.uint16)
+            pack(g[r0 * int(cols[t]):r0 * int(cols[t]) + k], seg, scale)
+            buf[dst:dst + k] = seg
+    return buf
+
+
 def bf16_round(x):
     """float32 -> bf16 bits, round to nearest even."""
     x = np.ascontiguousarray(x, dtype=np.float32)

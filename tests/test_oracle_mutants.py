@@ -1,9 +1,10 @@
 """Plant plausible mistakes in a copy of the oracle and check that its pins
 fail (CPU only).
 
-Each case rewrites one line of a temporary copy of ``oracle/oracle.cpp``
-(a flipped sign, a dropped term, a swapped operand, a wrong rounding or
-layout rule), rebuilds it there, and runs the pin test that must catch it.
+Each case rewrites one line of a temporary copy of ``oracle/oracle.cpp`` or
+``oracle/__init__.py`` (a flipped sign, a dropped term, a swapped operand, a
+wrong rounding or layout rule), rebuilds it there, and runs the pin test that
+must catch it.
 The real oracle is never modified.
 """
 import os
@@ -62,11 +63,29 @@ MUTANTS = {
                               "test_oracle_layout.py::test_literal_scan_equals_walk"),
 }
 
+# The same for the oracle's Python part (oracle/__init__.py).
+PY_MUTANTS = {
+    "rowwise_floor_rows": ("    q = (rows + m - 1) // m", "    q = rows // m",
+                           "test_oracle_rowwise.py::test_golden_rowwise_layout"),
+    "rowwise_inclusive_offsets": ("    off = np.concatenate([[0], np.cumsum(sizes)[:-1]]).astype(np.int64)",
+                                  "    off = (np.cumsum(sizes) - sizes[0]).astype(np.int64)",
+                                  "test_oracle_rowwise.py::test_golden_rowwise_layout"),
+    "rowwise_rank_minor": ("            src = r * C + int(off[t])", "            src = int(off[t]) * m + r",
+                           "test_oracle_rowwise.py::test_copy_out_inverts_copy_in"),
+    "rowwise_unscaled": ("            pack(g[r0 * int(cols[t]):r0 * int(cols[t]) + k], seg, scale)",
+                         "            pack(g[r0 * int(cols[t]):r0 * int(cols[t]) + k], seg, 1.0)",
+                         "test_oracle_rowwise.py::test_golden_rowwise_layout"),
+}
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
+
+ALL = {**{k: ("oracle.cpp",) + v for k, v in MUTANTS.items()},
+       **{k: ("__init__.py",) + v for k, v in PY_MUTANTS.items()}}
+
+
+@pytest.mark.parametrize("name", sorted(ALL))
 def test_pin_catches_planted_mistake(name, tmp_path):
-    orig, bad, pin = MUTANTS[name]
-    src = open(os.path.join(ROOT, "oracle", "oracle.cpp")).read()
+    fname, orig, bad, pin = ALL[name]
+    src = open(os.path.join(ROOT, "oracle", fname)).read()
     assert src.count(orig) == 1, f"mutation site of {name} not found once"
     work = tmp_path / "repo"
     os.makedirs(work / "tests")
@@ -74,10 +93,10 @@ def test_pin_catches_planted_mistake(name, tmp_path):
                     ignore=shutil.ignore_patterns("*.so", "__pycache__"))
     shutil.copytree(os.path.join(ROOT, "synth"), work / "synth",
                     ignore=shutil.ignore_patterns("__pycache__"))
-    for f in ("conftest.py", "test_oracle_adam.py", "test_oracle_layout.py"):
+    for f in ("conftest.py", "test_oracle_adam.py", "test_oracle_layout.py", "test_oracle_rowwise.py"):
         shutil.copy(os.path.join(ROOT, "tests", f), work / "tests" / f)
     shutil.copytree(os.path.join(ROOT, "tests", "golden"), work / "tests" / "golden")
-    (work / "oracle" / "oracle.cpp").write_text(src.replace(orig, bad))
+    (work / "oracle" / fname).write_text(src.replace(orig, bad))
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
                         "tests/" + pin], cwd=work, capture_output=True, text=True, timeout=600)
     assert r.returncode == 1 and "failed" in r.stdout, (
