@@ -40,13 +40,6 @@ using dbuf_detail::fail;
 
 extern "C" const char* dbuf_last_error(void) { return dbuf_detail::g_err.c_str(); }
 
-#define CUDA_TRY(call, what)                                                                  \
-    do {                                                                                      \
-        cudaError_t e_ = (call);                                                              \
-        if (e_ != cudaSuccess)                                                                \
-            return fail(DBUF_ECUDA, std::string(what) + ": " + cudaGetErrorString(e_));       \
-    } while (0)
-
 // ------------------------------------------------------------ work tables
 
 namespace {
@@ -191,7 +184,7 @@ dbuf_status check_device(const dbuf_t* db, const char* who) {
 }
 
 // Persistent grid of the step kernel on the current device: as many CTAs as
-// fit at once (two per SM with its shared-memory ring), never more than tiles.
+// fit at once (three per SM with its shared-memory ring), never more than tiles.
 dbuf_status step_grid_for(int device, size_t n_tiles, int* grid) {
     static bool attr_set[64] = {false};
     if (device >= 0 && device < 64 && !attr_set[device]) {

@@ -24,3 +24,12 @@ void set_error(const std::string& msg);
 dbuf_status fail(dbuf_status st, const std::string& msg);
 
 }  // namespace dbuf_detail
+
+// Return DBUF_ECUDA with the CUDA error text from a C-ABI function (CUDA
+// sources only).
+#define CUDA_TRY(call, what)                                                                            \
+    do {                                                                                                \
+        cudaError_t e_ = (call);                                                                        \
+        if (e_ != cudaSuccess)                                                                          \
+            return dbuf_detail::fail(DBUF_ECUDA, std::string(what) + ": " + cudaGetErrorString(e_));    \
+    } while (0)

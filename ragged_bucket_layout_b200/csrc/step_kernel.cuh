@@ -70,6 +70,7 @@ struct StepShared {
     float dqm[256], dqv[256];   // dequantisation steps of the old codes
     float qm[256], qv[256];     // quantisation factors of the new codes
     float red[2][kConsumerWarps];
+    uint32_t am1[2], ar1[2];    // single-block tiles: absmax, double-buffered by tile parity
     int32_t go[2];
 };
 
@@ -191,9 +192,10 @@ __device__ __forceinline__ void sqrt_vec(const float2* v, float2* r) {
     }
 }
 
+template <bool FAST>
 __device__ __forceinline__ float2 new_p2(float2 p, float2 m, float2 r, const StepC2& c) {
     const float2 d = sum_of(r, c.eps_hat);  // r ends a square-root sequence: keep the add scalar
-    const float2 u = make_float2(__fdiv_rn(m.x, d.x), __fdiv_rn(m.y, d.y));
+    const float2 u = FAST ? div2_fast(m, d) : make_float2(__fdiv_rn(m.x, d.x), __fdiv_rn(m.y, d.y));
     return diff_of(mul2(p, c.decay), mul2(c.step_hat, u));
 }
 
@@ -373,19 +375,43 @@ __device__ __forceinline__ void mr8(const In8& x, float dqm, float dqv, const St
     }
 }
 
-// Update of one vector whose elements share dqm/dqv (one block).
+// Update of one vector whose elements share dqm/dqv (one block); am, ar
+// receive the vector's max |m| and max sqrt(v).  The division takes the
+// fast sequence when the whole vector lies in its range: d = sqrt(v) + eps
+// >= eps >= 2^-60 and sqrt(v) <= 2^64 bound d, and |m| is bounded on both
+// sides (a zero m takes the IEEE path).
 template <bool FULL>
 __device__ __forceinline__ void update8(const unsigned char* st, int li, int lo, int hi, float dqm, float dqv,
-                                        const StepC2& c, const Out& o, float* m, float* r) {
+                                        const StepC2& c, const Out& o, float* m, float* r, float& am, float& ar) {
     In8 x;
     load8<FULL>(x, st, li, lo, hi, true);
     mr8(x, dqm, dqv, c, m, r);
+    float mn = fabsf(m[0]);
+    am = 0.f;
+    ar = 0.f;
 #pragma unroll
-    for (int j = 0; j < kV / 2; ++j) {
-        const float2 pn = new_p2(make_float2(x.p[2 * j], x.p[2 * j + 1]), make_float2(m[2 * j], m[2 * j + 1]),
-                                 make_float2(r[2 * j], r[2 * j + 1]), c);
-        x.p[2 * j] = pn.x;
-        x.p[2 * j + 1] = pn.y;
+    for (int i = 0; i < kV; ++i) {
+        am = fmaxf(am, fabsf(m[i]));
+        mn = fminf(mn, fabsf(m[i]));
+        ar = fmaxf(ar, r[i]);
+    }
+    const bool fast = am <= kDivMaxA && mn >= kDivMinA && ar <= 0.5f * kDivMaxD && c.eps_hat.x >= kDivMinD;
+    if (fast) {
+#pragma unroll
+        for (int j = 0; j < kV / 2; ++j) {
+            const float2 pn = new_p2<true>(make_float2(x.p[2 * j], x.p[2 * j + 1]),
+                                           make_float2(m[2 * j], m[2 * j + 1]), make_float2(r[2 * j], r[2 * j + 1]), c);
+            x.p[2 * j] = pn.x;
+            x.p[2 * j + 1] = pn.y;
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < kV / 2; ++j) {
+            const float2 pn = new_p2<false>(make_float2(x.p[2 * j], x.p[2 * j + 1]),
+                                            make_float2(m[2 * j], m[2 * j + 1]), make_float2(r[2 * j], r[2 * j + 1]), c);
+            x.p[2 * j] = pn.x;
+            x.p[2 * j + 1] = pn.y;
+        }
     }
     store_p8<FULL>(x.p, li, lo, hi, o);
 }
@@ -515,13 +541,78 @@ __device__ void step_producer(const Tile* __restrict__ tiles, int64_t n_tiles, i
     }
 }
 
-// Kinds of whole-block tiles, fixed per tile.
-enum : int { W_SINGLE = 0, W_MULTI8 = 1, W_MIXED = 2 };
+// A tile that is one block (the common case: 1-row blocks up to 4096
+// elements).  Every consumer computes the block's dequantisation and
+// quantisation factors itself, so only the absmax needs a barrier.  The
+// absmax words alternate between two slots by tile parity: the slot of the
+// next single-block tile is cleared here, after every reader of its last use
+// has passed this tile's first barrier.
+__device__ void single_tile(const Tile& t, unsigned char* st, StepShared& sh, uint32_t par, float* master,
+                            uint16_t* param, int8_t* mq, uint8_t* vq, float2* scales, const StepC& c) {
+    const int tid = threadIdx.x;
+    const float2 sc = reinterpret_cast<const float2*>(st + kOffS)[t.blk0 & 1];
+    const float2 dq = dequant_steps(sc);
+    const float dqm = dq.x, dqv = dq.y;
+    if (tid == 0) {
+        sh.am1[par ^ 1u] = 0u;
+        sh.ar1[par ^ 1u] = 0u;
+    }
+    const int64_t a0 = t.e0 & ~int64_t(kAlign - 1);
+    const Out o{master + a0, param + a0, mq + a0, vq + a0};
+    const int lo = (int)(t.e0 - a0), hi = lo + (int)t.n;
+    const StepC2 c2 = pairs_of(c);
+    float am = 0.f, ar = 0.f;
+#pragma unroll
+    for (int j = 0; j < kSub; ++j) {
+        const int li = j * (kConsumers * kV) + kV * tid;
+        if (!(li < hi && li + kV > lo)) continue;
+        float m[kV], r[kV], vm, vr;
+        if (li >= lo && li + kV <= hi)
+            update8<true>(st, li, lo, hi, dqm, dqv, c2, o, m, r, vm, vr);
+        else
+            update8<false>(st, li, lo, hi, dqm, dqv, c2, o, m, r, vm, vr);
+        am = fmaxf(am, vm);
+        ar = fmaxf(ar, vr);
+        stash_mr(st, li, m, r);
+    }
+    warp_max2(am, ar);
+    if ((tid & 31) == 0) {
+        atomicMax(&sh.am1[par], __float_as_uint(am));
+        atomicMax(&sh.ar1[par], __float_as_uint(ar));
+    }
+    named_sync(kBarCons, kConsumers);
+    const float AMm = __uint_as_float(sh.am1[par]), AMr = __uint_as_float(sh.ar1[par]);
+    float qm[kV], qv[kV];
+    {
+        const float2 qf = quant_factors(make_float2(AMm, AMr));
+        const float q1 = qf.x, q2 = qf.y;
+#pragma unroll
+        for (int i = 0; i < kV; ++i) {
+            qm[i] = q1;
+            qv[i] = q2;
+        }
+    }
+    if (tid == 0) scales[t.blk0] = make_float2(AMm, AMr);
+#pragma unroll
+    for (int j = 0; j < kSub; ++j) {
+        const int li = j * (kConsumers * kV) + kV * tid;
+        if (!(li < hi && li + kV > lo)) continue;
+        float m[kV], r[kV];
+        unstash_mr(st, li, m, r);
+        if (li >= lo && li + kV <= hi)
+            store_codes8<true>(m, r, qm, qv, li, lo, hi, o);
+        else
+            store_codes8<false>(m, r, qm, qv, li, lo, hi, o);
+    }
+}
 
-// Whole blocks: phase 1 updates the weights and parks m, sqrt(v) in the
-// stage; block maxima meet in shared memory; phase 2 writes the codes.
-//   W_SINGLE: one block.  W_MULTI8: blocks of a multiple of 8 elements, so
-//   each vector lies in one block, found as umulhi(x, magic) = x / b.
+// Kinds of multi-block tiles, fixed per tile.
+enum : int { W_MULTI8 = 1, W_MIXED = 2 };
+
+// Several whole blocks: phase 1 updates the weights and parks m, sqrt(v) in
+// the stage; block maxima meet in shared memory; phase 2 writes the codes.
+//   W_MULTI8: blocks of a multiple of 8 elements, so each vector lies in one
+//   block, found as umulhi(x, magic) = x / b.
 //   W_MIXED: blocks not a multiple of 8 elements, per-element block numbers (rare).
 template <int MODE>
 __device__ void whole_tile(const Tile& t, unsigned char* st, StepShared& sh, float* master, uint16_t* param,
@@ -530,8 +621,9 @@ __device__ void whole_tile(const Tile& t, unsigned char* st, StepShared& sh, flo
     const int nb = t.nblk;
     if (tid < nb) {
         const float2 sc = reinterpret_cast<const float2*>(st + kOffS)[(t.blk0 & 1) + tid];
-        sh.dqm[tid] = __fdiv_rn(sc.x, 127.f);
-        sh.dqv[tid] = __fdiv_rn(sc.y, 255.f);
+        const float2 dq = dequant_steps(sc);
+        sh.dqm[tid] = dq.x;
+        sh.dqv[tid] = dq.y;
         sh.am[tid] = 0u;
         sh.ar[tid] = 0u;
     }
@@ -542,40 +634,21 @@ __device__ void whole_tile(const Tile& t, unsigned char* st, StepShared& sh, flo
     const int lo = (int)(t.e0 - a0), hi = lo + (int)t.n;  // local range of the tile's elements
     const StepC2 c2 = pairs_of(c);
     const uint32_t b = (uint32_t)t.b, magic = t.magic;
-    float am1 = 0.f, ar1 = 0.f;
 #pragma unroll
     for (int j = 0; j < kSub; ++j) {
         const int li = j * (kConsumers * kV) + kV * tid;
         const bool any = li < hi && li + kV > lo;
         const bool full = li >= lo && li + kV <= hi;
         float m[kV], r[kV];
-        if (MODE == W_SINGLE) {
-            if (any) {
-                if (full)
-                    update8<true>(st, li, lo, hi, sh.dqm[0], sh.dqv[0], c2, o, m, r);
-                else
-                    update8<false>(st, li, lo, hi, sh.dqm[0], sh.dqv[0], c2, o, m, r);
-#pragma unroll
-                for (int i = 0; i < kV; ++i) {
-                    am1 = fmaxf(am1, fabsf(m[i]));
-                    ar1 = fmaxf(ar1, r[i]);
-                }
-                stash_mr(st, li, m, r);
-            }
-        } else if (MODE == W_MULTI8) {
+        if (MODE == W_MULTI8) {
             int key = -1;
             float am = 0.f, ar = 0.f;
             if (any) {
                 key = (int)__umulhi((uint32_t)(max(li, lo) - lo), magic);
                 if (full)
-                    update8<true>(st, li, lo, hi, sh.dqm[key], sh.dqv[key], c2, o, m, r);
+                    update8<true>(st, li, lo, hi, sh.dqm[key], sh.dqv[key], c2, o, m, r, am, ar);
                 else
-                    update8<false>(st, li, lo, hi, sh.dqm[key], sh.dqv[key], c2, o, m, r);
-#pragma unroll
-                for (int i = 0; i < kV; ++i) {
-                    am = fmaxf(am, fabsf(m[i]));
-                    ar = fmaxf(ar, r[i]);
-                }
+                    update8<false>(st, li, lo, hi, sh.dqm[key], sh.dqv[key], c2, o, m, r, am, ar);
                 stash_mr(st, li, m, r);
             }
             block_max_to_smem(key, am, ar, sh);
@@ -600,12 +673,12 @@ __device__ void whole_tile(const Tile& t, unsigned char* st, StepShared& sh, flo
             }
         }
     }
-    if (MODE == W_SINGLE) block_max_to_smem(0, am1, ar1, sh);
     named_sync(kBarCons, kConsumers);
     if (tid < nb) {
         const float AMm = __uint_as_float(sh.am[tid]), AMr = __uint_as_float(sh.ar[tid]);
-        sh.qm[tid] = AMm > 0.f ? __fdiv_rn(127.f, AMm) : 0.f;
-        sh.qv[tid] = AMr > 0.f ? __fdiv_rn(255.f, AMr) : 0.f;
+        const float2 qf = quant_factors(make_float2(AMm, AMr));
+        sh.qm[tid] = qf.x;
+        sh.qv[tid] = qf.y;
         scales[t.blk0 + tid] = make_float2(AMm, AMr);
     }
     named_sync(kBarCons, kConsumers);
@@ -625,7 +698,7 @@ __device__ void whole_tile(const Tile& t, unsigned char* st, StepShared& sh, flo
                 qv[i] = sh.qv[blk];
             }
         } else {
-            const int key = MODE == W_SINGLE ? 0 : (int)__umulhi((uint32_t)(max(li, lo) - lo), magic);
+            const int key = (int)__umulhi((uint32_t)(max(li, lo) - lo), magic);
             const float q1 = sh.qm[key], q2 = sh.qv[key];
 #pragma unroll
             for (int i = 0; i < kV; ++i) {
@@ -648,7 +721,8 @@ __device__ bool large_tile(const Tile& t, uint32_t& k, unsigned char* stages, St
                            int32_t* status) {
     const int tid = threadIdx.x;
     const float2 sc = scales[t.blk0];
-    const float dqm = __fdiv_rn(sc.x, 127.f), dqv = __fdiv_rn(sc.y, 255.f);
+    const float2 dq = dequant_steps(sc);
+    const float dqm = dq.x, dqv = dq.y;
     const int64_t a0 = t.e0 & ~int64_t(kAlign - 1);
     const int64_t nch = large_chunks(t);
     const StepC2 c2 = pairs_of(c);
@@ -664,16 +738,13 @@ __device__ bool large_tile(const Tile& t, uint32_t& k, unsigned char* stages, St
         for (int j = 0; j < kSub; ++j) {
             const int li = j * (kConsumers * kV) + kV * tid;
             if (!(li < hi && li + kV > lo)) continue;
-            float m[kV], r[kV];
+            float m[kV], r[kV], vm, vr;
             if (li >= lo && li + kV <= hi)
-                update8<true>(st, li, lo, hi, dqm, dqv, c2, o, m, r);
+                update8<true>(st, li, lo, hi, dqm, dqv, c2, o, m, r, vm, vr);
             else
-                update8<false>(st, li, lo, hi, dqm, dqv, c2, o, m, r);
-#pragma unroll
-            for (int i = 0; i < kV; ++i) {
-                am = fmaxf(am, fabsf(m[i]));
-                ar = fmaxf(ar, r[i]);
-            }
+                update8<false>(st, li, lo, hi, dqm, dqv, c2, o, m, r, vm, vr);
+            am = fmaxf(am, vm);
+            ar = fmaxf(ar, vr);
         }
         release_stage(sh, k);
         ++k;
@@ -691,8 +762,9 @@ __device__ bool large_tile(const Tile& t, uint32_t& k, unsigned char* stages, St
             a = fmaxf(a, sh.red[0][w]);
             q = fmaxf(q, sh.red[1][w]);
         }
-        sh.qm[0] = a > 0.f ? __fdiv_rn(127.f, a) : 0.f;
-        sh.qv[0] = q > 0.f ? __fdiv_rn(255.f, q) : 0.f;
+        const float2 qf = quant_factors(make_float2(a, q));
+        sh.qm[0] = qf.x;
+        sh.qv[0] = qf.y;
         scales[t.blk0] = make_float2(a, q);
     }
     named_sync(kBarCons, kConsumers);
@@ -762,6 +834,7 @@ __global__ void __launch_bounds__(kStepThreads, DBUF_STEP_MIN_CTAS)
             mbar_init(&sh.empty[s], kConsumerWarps);
         }
         fence_barrier_init();
+        sh.am1[0] = sh.am1[1] = sh.ar1[0] = sh.ar1[1] = 0u;
     }
     __syncthreads();
     if (tid >= kConsumers) {  // producer warp: one lane issues all copies
@@ -769,7 +842,7 @@ __global__ void __launch_bounds__(kStepThreads, DBUF_STEP_MIN_CTAS)
             step_producer(tiles, n_tiles, bucket, n_blocks, master, grad, mq, vq, scales, stages, sh, status);
         return;
     }
-    uint32_t k = 0;
+    uint32_t k = 0, nsingle = 0;
     // The next table entry is loaded one tile ahead, so its latency hides
     // behind the current tile.
     Tile nxt;
@@ -786,9 +859,10 @@ __global__ void __launch_bounds__(kStepThreads, DBUF_STEP_MIN_CTAS)
         } else if (t.kind == TILE_WHOLE) {
             if (!wait_stage(sh, k, status)) return;
             unsigned char* st = stages + (k % kStages) * kStageBytes;
-            if (t.nblk == 1)
-                whole_tile<W_SINGLE>(t, st, sh, master, param, mq, vq, scales, c);
-            else if ((t.b & 7) == 0)
+            if (t.nblk == 1) {
+                single_tile(t, st, sh, nsingle & 1u, master, param, mq, vq, scales, c);
+                ++nsingle;
+            } else if ((t.b & 7) == 0)
                 whole_tile<W_MULTI8>(t, st, sh, master, param, mq, vq, scales, c);
             else
                 whole_tile<W_MIXED>(t, st, sh, master, param, mq, vq, scales, c);
