@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-copy-in", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--graph-steps", type=int, default=10,
+                    help="steps per CUDA graph for the launch-overhead-free figure (0: skip)")
     return ap.parse_args()
 
 
@@ -71,7 +73,7 @@ def measured_peak():
 
 def kernel_source_hash():
     h = hashlib.sha256()
-    for f in ("dbuf.cu", "internal.h", "step_kernel.cuh", "tma.cuh", "tables.h"):
+    for f in ("dbuf.cu", "internal.h", "step_kernel.cuh", "fastmath.cuh", "tma.cuh", "tables.h"):
         h.update(open(os.path.join(ROOT, "ragged_bucket_layout_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -319,6 +321,32 @@ def run_ours(args):
     value, per_step_ms = job_throughput(ms, args.steps, world, stats["step_bytes"])
     kernel_gbs = stats["step_bytes"] / (ms_local / args.steps * 1e-3) / 1e9
 
+    # ---- the same steps replayed from a CUDA graph (no per-launch host
+    # overhead; matters for small buckets).  The graph holds steps
+    # t+1..t+G with their hyper-parameters fixed at capture.
+    graph = None
+    if args.graph_steps > 0:
+        G = args.graph_steps
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(G):
+                D.step(hp_at(step_no + 1 + i), gscale)
+        step_no += G
+        for _ in range(3):
+            g.replay()
+        reps = max(3, min(100, args.steps // G))
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            g0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            g1.record(stream)
+        g1.synchronize()
+        gms = max_over_ranks(g0.elapsed_time(g1), dist, "cuda") / (reps * G)
+        graph = {"steps_per_graph": G, "replays": reps, "ms_per_step": gms,
+                 "value": world * stats["step_bytes"] / (gms * 1e-3) / 1e9, "unit": UNIT}
+        del g
+
     # ---- end to end through the host-buffer entry point
     S = info["bucket"]
     e2e = None
@@ -393,7 +421,34 @@ def run_ours(args):
             "accumulate_gbs": 6 * stats["params"] / (acc_ms * 1e-3) / 1e9, "accumulate_ms": acc_ms,
             "grad_norm_gbs": 2 * stats["bucket"] / (norm_ms * 1e-3) / 1e9, "grad_norm_ms": norm_ms,
             "clipped_step_ms": clip_ms, "clipped_step_gbs": (stats["step_bytes"] + 2 * stats["bucket"]) / (clip_ms * 1e-3) / 1e9}
-        del sep
+        # Row-wise (FSDP2-style) baseline: the interleaved copy-in before the
+        # ReduceScatter and copy-out after the AllGather that the bucket
+        # layout does without, on the same tensors and m.
+        R = rb.Rowwise(r, c, w.m, stream=stream)
+        flat = torch.empty(w.m * R.chunk, dtype=torch.bfloat16, device="cuda")
+        outs = [torch.empty_like(x) for x in sep]
+        with torch.cuda.stream(stream):
+            R.copy_in(sep, gscale, flat, stream=stream)
+            R.copy_out(flat, outs, stream=stream)
+            r0, r1, r2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            r0.record(stream)
+            for _ in range(reps):
+                R.copy_in(sep, gscale, flat, stream=stream)
+            r1.record(stream)
+            for _ in range(reps):
+                R.copy_out(flat, outs, stream=stream)
+            r2.record(stream)
+        r2.synchronize()
+        if R.status(stream=stream) != 0:
+            raise RuntimeError("row-wise copy status word set")
+        in_ms, out_ms = r0.elapsed_time(r1) / reps, r1.elapsed_time(r2) / reps
+        copy_in["rowwise_baseline"] = {
+            "copy_in_gbs": stats["copy_in_bytes"] / (in_ms * 1e-3) / 1e9, "copy_in_ms": in_ms,
+            "copy_out_gbs": stats["copy_in_bytes"] / (out_ms * 1e-3) / 1e9, "copy_out_ms": out_ms,
+            "gathered_elems": w.m * R.chunk,
+            "copies_vs_step": (in_ms + out_ms) / (ms_local / args.steps)}
+        R.close()
+        del sep, flat, outs
 
     peak, peak_src = measured_peak()
     roof = {"bound": "hbm", "achieved": kernel_gbs, "peak": peak, "unit": "GB/s", "frac": kernel_gbs / peak,
@@ -415,7 +470,7 @@ def run_ours(args):
                    "parallelism": f"dp{world} (one bucket per rank, no data-path collective)"},
         "params_per_s": world * stats["params"] / (per_step_ms * 1e-3),
         "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps,
-        "clocks": clk.summary(), "copy_in": copy_in,
+        "clocks": clk.summary(), "cuda_graph": graph, "copy_in": copy_in,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

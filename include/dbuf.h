@@ -237,6 +237,64 @@ dbuf_status dbuf_clear_device_status(dbuf_t* db, void* stream);
 
 void dbuf_destroy(dbuf_t* db); /* NULL is a no-op; frees only what it allocated */
 
+/* ------------------------------------------------ row-wise baseline layout
+ *
+ * The layout RaggedShard replaces, for measuring what it saves: row-wise even
+ * sharding as in FSDP2 / Megatron-FSDP (veScale-FSDP pages, comparison of
+ * sharding formats; section on the importance of zero-copy communication:
+ * per-parameter copy-in and copy-out with interleaved addresses cost 12-31%
+ * of communication time).  Tensor i (rows_i x cols_i, row-major bf16) is
+ * cut along dim 0 into m shards of q_i = ceil(rows_i / m) rows, the last
+ * ones shorter or empty, each padded to q_i rows in the communication
+ * buffer.  Rank r's chunk concatenates its padded shards of tensors 0..n-1;
+ * a gathered buffer holds the m chunks in rank order, m * chunk_elems bf16
+ * elements.  The k of each descriptor is ignored (it must still be valid). */
+typedef struct dbuf_rowwise_s dbuf_rowwise_t;
+
+/* The layout alone, on the host (no CUDA call): chunk_elems, and when not
+ * NULL shard_rows[n] (q_i) and offsets[n] (element offset of tensor i's
+ * shard in a chunk).  DBUF_EINVAL for n < 1 or m < 1 or an invalid
+ * descriptor. */
+dbuf_status dbuf_rowwise_layout(const dbuf_tensor_desc* tensors, int32_t n, int32_t m, int64_t* chunk_elems,
+                                int64_t* shard_rows, int64_t* offsets);
+
+/* Build the layout and its device copy table (one cudaMalloc, freed by
+ * dbuf_rowwise_destroy; the table is copied in on `stream`, and the call
+ * waits for that copy).  DBUF_EINVAL for n < 1 or m < 1 or an invalid
+ * descriptor. */
+dbuf_status dbuf_rowwise_create(const dbuf_tensor_desc* tensors, int32_t n, int32_t m, void* stream,
+                                dbuf_rowwise_t** out);
+
+/* chunk_elems: elements per rank chunk.  shard_rows[n] (q_i) and
+ * offsets[n] (element offset of tensor i's shard in a chunk) are filled when
+ * not NULL (host arrays). */
+dbuf_status dbuf_rowwise_info(const dbuf_rowwise_t* rw, int64_t* chunk_elems, int64_t* shard_rows,
+                              int64_t* offsets);
+
+/* Interleaved copy-out after an AllGather: for every tensor i and rank r,
+ *   params_bf16[i][r*q_i*cols_i + j] = gathered_bf16[r*chunk + offsets_i + j],
+ *   j < (min(rows_i, (r+1)*q_i) - r*q_i) * cols_i  (bits copied as they are).
+ * gathered_bf16: device, m * chunk_elems elements.  params_bf16[n]: device
+ * pointers in tensor order (host array, read during the call).  Any 2-byte
+ * alignment; the memory must stay valid until the copy completes on
+ * `stream`. */
+dbuf_status dbuf_rowwise_copy_out(dbuf_rowwise_t* rw, const void* gathered_bf16, void* const* params_bf16,
+                                  void* stream);
+
+/* Interleaved copy-in before a ReduceScatter: the inverse placement of
+ * dbuf_rowwise_copy_out with every element scaled,
+ *   rs_input_bf16[r*chunk + offsets_i + j] = bf16(float(grads_bf16[i][r*q_i*cols_i + j]) * scale),
+ * and the padding rows of every shard set to 0.  rs_input_bf16: device,
+ * m * chunk_elems elements.  Arguments and lifetimes as above. */
+dbuf_status dbuf_rowwise_copy_in(dbuf_rowwise_t* rw, const void* const* grads_bf16, float scale,
+                                 void* rs_input_bf16, void* stream);
+
+/* Status word of the copy kernels, read after the work queued on `stream`
+ * (waits for it): 0 = fine, 2 = a malformed copy-table entry was skipped. */
+dbuf_status dbuf_rowwise_status(dbuf_rowwise_t* rw, int32_t* code, void* stream);
+
+void dbuf_rowwise_destroy(dbuf_rowwise_t* rw); /* NULL is a no-op */
+
 /* Message of the last failure on this host thread ("" if none). */
 const char* dbuf_last_error(void);
 

@@ -76,6 +76,13 @@ _SIGS = {
     "dbuf_work_table": (ctypes.c_int, [_P, ctypes.POINTER(dbuf_work_item), _i64, _pi64]),
     "dbuf_destroy": (None, [_P]),
     "dbuf_last_error": (ctypes.c_char_p, []),
+    "dbuf_rowwise_layout": (ctypes.c_int, [ctypes.POINTER(dbuf_tensor_desc), _i32, _i32, _pi64, _pi64, _pi64]),
+    "dbuf_rowwise_create": (ctypes.c_int, [ctypes.POINTER(dbuf_tensor_desc), _i32, _i32, _P, _PP]),
+    "dbuf_rowwise_info": (ctypes.c_int, [_P, _pi64, _pi64, _pi64]),
+    "dbuf_rowwise_copy_out": (ctypes.c_int, [_P, _P, _PP, _P]),
+    "dbuf_rowwise_copy_in": (ctypes.c_int, [_P, _PP, _f32, _P, _P]),
+    "dbuf_rowwise_status": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int32), _P]),
+    "dbuf_rowwise_destroy": (None, [_P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -110,10 +117,11 @@ class Plan:
     def __init__(self, handle, n):
         self.handle = handle
         self.n = n
+        self._free = _lib.dbuf_plan_free   # held here: module globals may be gone at interpreter exit
 
     def __del__(self):
         if getattr(self, "handle", None):
-            _lib.dbuf_plan_free(self.handle)
+            self._free(self.handle)
             self.handle = None
 
 
@@ -235,6 +243,66 @@ def dbuf_clear_device_status(db, stream=None):
     _check(_lib.dbuf_clear_device_status(db, _stream(stream)))
 
 
+# --------------------------------------------- row-wise baseline layout
+
+def dbuf_rowwise_layout(rows, cols, m):
+    """Row-wise (FSDP2-style) layout on the host: (chunk_elems, shard_rows, offsets)."""
+    n = len(rows)
+    descs = (dbuf_tensor_desc * max(n, 1))(*[dbuf_tensor_desc(int(r), int(c), 1) for r, c in zip(rows, cols)])
+    chunk = ctypes.c_int64()
+    q = (ctypes.c_int64 * max(n, 1))()
+    off = (ctypes.c_int64 * max(n, 1))()
+    _check(_lib.dbuf_rowwise_layout(descs, n, int(m), ctypes.byref(chunk), q, off))
+    return chunk.value, list(q[:n]), list(off[:n])
+
+
+class Rowwise:
+    """Row-wise (FSDP2-style) sharded layout of a tensor list and its
+    interleaved copy-in / copy-out (the copies the bucket layout avoids).
+    Owner of a dbuf_rowwise_t; all work goes through the C-ABI."""
+
+    def __init__(self, rows, cols, m, stream=None):
+        n = len(rows)
+        descs = (dbuf_tensor_desc * max(n, 1))(*[dbuf_tensor_desc(int(r), int(c), 1) for r, c in zip(rows, cols)])
+        h = ctypes.c_void_p()
+        _check(_lib.dbuf_rowwise_create(descs, n, int(m), _stream(stream), ctypes.byref(h)))
+        self.handle, self.n, self.m = h, n, int(m)
+        self._destroy = _lib.dbuf_rowwise_destroy   # held here: module globals may be gone at interpreter exit
+        chunk = ctypes.c_int64()
+        q = (ctypes.c_int64 * max(n, 1))()
+        off = (ctypes.c_int64 * max(n, 1))()
+        _check(_lib.dbuf_rowwise_info(self.handle, ctypes.byref(chunk), q, off))
+        self.chunk, self.shard_rows, self.offsets = chunk.value, list(q[:n]), list(off[:n])
+
+    def close(self):
+        if getattr(self, "handle", None):
+            self._destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        self.close()
+
+    @staticmethod
+    def _ptrs(ts):
+        return (ctypes.c_void_p * max(len(ts), 1))(*[int(t.data_ptr()) if hasattr(t, "data_ptr") else int(t)
+                                                     for t in ts])
+
+    def copy_out(self, gathered, params, stream=None):
+        """params[i] <- tensor i's rows from the m chunks of `gathered`."""
+        _check(_lib.dbuf_rowwise_copy_out(self.handle, int(gathered.data_ptr()), self._ptrs(params),
+                                          _stream(stream)))
+
+    def copy_in(self, grads, scale, rs_input, stream=None):
+        """rs_input <- bf16(float(g) * scale) of every tensor at its ranks' shards; padding rows 0."""
+        _check(_lib.dbuf_rowwise_copy_in(self.handle, self._ptrs(grads), float(scale), int(rs_input.data_ptr()),
+                                         _stream(stream)))
+
+    def status(self, stream=None):
+        code = ctypes.c_int32()
+        _check(_lib.dbuf_rowwise_status(self.handle, ctypes.byref(code), _stream(stream)))
+        return code.value
+
+
 # ----------------------------------------------------- PyTorch-owned buckets
 
 _DTYPES = None
@@ -263,11 +331,12 @@ class DBuffer:
         nbytes = dbuf_required_bytes(plan)
         self.base = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
         self.stream = stream if stream is not None else torch.cuda.current_stream(self.base.device)
+        self._destroy = _lib.dbuf_destroy   # held here: module globals may be gone at interpreter exit
         self.handle = dbuf_create(plan, self.base.data_ptr(), self.base.numel(), self.stream)
 
     def close(self):
         if getattr(self, "handle", None):
-            dbuf_destroy(self.handle)
+            self._destroy(self.handle)
             self.handle = None
 
     def __del__(self):

@@ -7,8 +7,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libdbuf.so")
-SOURCES = [os.path.join(CSRC, f) for f in ("dbuf.cu", "planner.cpp")]
-HEADERS = [os.path.join(CSRC, "internal.h"), os.path.join(ROOT, "include", "dbuf.h")]
+SOURCES = [os.path.join(CSRC, f) for f in ("dbuf.cu", "rowwise.cu", "planner.cpp")]
+HEADERS = [os.path.join(CSRC, f) for f in sorted(os.listdir(CSRC)) if f.endswith((".h", ".cuh"))] + [
+    os.path.join(ROOT, "include", "dbuf.h")]
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",

@@ -83,16 +83,17 @@ def llama_layer(m=8):
                     description="Llama layer h=4096, GQA 32q/8kv, SwiGLU 14336; 1-row blocks; m=8")
 
 
-def moe_layer(m=64):
+def moe_layer(m=64, experts=32):
     ts = []
-    for e in range(32):
+    for e in range(experts):
         ts.append(TensorSpec(f"e{e}.gate_up", 5760, 2880, 16))
         ts.append(TensorSpec(f"e{e}.down", 2880, 2880, 16))
     ts.append(TensorSpec("router", 32, 2880, 1))
     ts += [TensorSpec("attn_q", 4096, 2880, 1), TensorSpec("attn_o", 4096, 2880, 1),
            TensorSpec("attn_k", 512, 2880, 1), TensorSpec("attn_v", 512, 2880, 1)]
-    return Workload(f"moe_layer_m{m}", ts, m=m, seed=2, steps=10,
-                    description="MoE layer h=2880, 32 experts (gate_up 5760x2880, down 2880x2880, "
+    name = f"moe_layer_m{m}" if experts == 32 else f"moe_layer_{experts}e_m{m}"
+    return Workload(name, ts, m=m, seed=2, steps=10,
+                    description=f"MoE layer h=2880, {experts} experts (gate_up 5760x2880, down 2880x2880, "
                                 "16-row blocks), router, attention (1-row blocks)")
 
 
@@ -166,6 +167,7 @@ _BUILDERS = {
     "tiny_m4": lambda: tiny(4),
     "llama_layer_m8": lambda: llama_layer(8),
     "moe_layer_m64": lambda: moe_layer(64),
+    "moe_layer_4e_m64": lambda: moe_layer(64, experts=4),   # profiling-size MoE bucket (1.9 GB moved per step)
     "ragged_stress_m8": lambda: ragged_stress(8),
     "ragged_stress_m128": lambda: ragged_stress(128),
     "ragged_stress_m1024": lambda: ragged_stress(1024),

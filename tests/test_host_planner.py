@@ -201,3 +201,19 @@ def test_block_index_reciprocal_is_exact():
     for b in range(2, 4097):
         magic = np.uint64(((1 << 32) + b - 1) // b)
         assert np.array_equal((x * magic) >> np.uint64(32), x // np.uint64(b)), b
+
+
+@pytest.mark.parametrize("m", [1, 2, 3, 8, 64, 1000])
+def test_rowwise_layout_matches_oracle(m):
+    w = synth.workload("ragged_mix_m4")
+    r, c, _ = w.arrays()
+    chunk, q, off = rb.dbuf_rowwise_layout(r, c, m)
+    oq, ooff, oc = oracle.rowwise_layout(r, c, m)
+    assert chunk == oc and q == oq.tolist() and off == ooff.tolist()
+
+
+def test_rowwise_layout_rejects_invalid():
+    for rows, cols, m in (([0], [3], 2), ([4], [0], 2), ([4], [3], 0), ([], [], 2)):
+        with pytest.raises(rb.DbufError) as e:
+            rb.dbuf_rowwise_layout(rows, cols, m)
+        assert e.value.status == rb.DBUF_EINVAL
