@@ -52,6 +52,9 @@ def _load():
     lib.orc_adam8_step.restype = None
     lib.orc_adam8_step.argtypes = [i64, P, P, P, P, P, P, P, P, P, P,
                                    f32, f32, f32, f32, f32, i64, f32, i32]
+    lib.orc_adam8_step_tiles.restype = None
+    lib.orc_adam8_step_tiles.argtypes = [i64, P, P, P, P, P, P, P, P, P, P, P, P,
+                                         f32, f32, f32, f32, f32, i64, f32, i32]
     lib.orc_step_scalars.restype = None
     lib.orc_step_scalars.argtypes = [f32, f32, f32, f32, f32, i64, P]
     lib.orc_pack.restype = None
@@ -154,6 +157,32 @@ def blocks(rows, cols, k, offsets):
     if not starts:
         return np.zeros(0, np.int64), np.zeros(0, np.int64)
     return np.concatenate(starts), np.concatenate(lens)
+
+
+def tiles(rows, cols, k, block_cols, offsets):
+    """Quantisation blocks of a planned bucket when a tensor's blocks are
+    k rows x block_cols columns (the 2-D 32x32 blocks the 8-bit Adam case
+    study allows per parameter; block_cols = 0, or >= cols, means whole
+    rows).  Numbered in bucket order: tensors by ascending offset, row blocks
+    top to bottom, column tiles left to right inside a row block; the last
+    row block and the last column tile may be smaller.  Returns int64 arrays
+    (base, trows, width, stride): tile j covers elements
+    base + r * stride + c for r < trows, c < width."""
+    rows, cols, k, off = _i64(rows), _i64(cols), _i64(k), _i64(offsets)
+    bc = _i64(block_cols) if block_cols is not None else np.zeros_like(rows)
+    base, trows, width, stride = [], [], [], []
+    for i in np.argsort(off, kind="stable"):
+        R, C, K = int(rows[i]), int(cols[i]), int(k[i])
+        W = C if int(bc[i]) <= 0 or int(bc[i]) >= C else int(bc[i])
+        for r0 in range(0, R, K):
+            nr = min(K, R - r0)
+            for c0 in range(0, C, W):
+                base.append(int(off[i]) + r0 * C + c0)
+                trows.append(nr)
+                width.append(min(W, C - c0))
+                stride.append(C)
+    mk = lambda a: np.asarray(a, dtype=np.int64)
+    return mk(base), mk(trows), mk(width), mk(stride)
 
 
 def padding_mask(rows, cols, offsets, bucket):
@@ -301,6 +330,26 @@ def bf16_round(x):
     return out
 
 
+def adam8_step_tiles(base, trows, width, stride, sidx, p, g_bits, mq, vq, scale_m, scale_v, pb_bits, hp, t,
+                     grad_scale, threads=1):
+    """Block-wise 8-bit Adam over 2-D tiles (see tiles()), in place: each
+    tile is quantised as one block, as adam8_step does for a contiguous one."""
+    base, trows, width, stride, sidx = _i64(base), _i64(trows), _i64(width), _i64(stride), _i64(sidx)
+    assert p.dtype == np.float32 and g_bits.dtype == np.uint16 and pb_bits.dtype == np.uint16
+    assert mq.dtype == np.int8 and vq.dtype == np.uint8
+    assert scale_m.dtype == np.float32 and scale_v.dtype == np.float32
+    for a in (p, g_bits, mq, vq, scale_m, scale_v, pb_bits):
+        assert a.flags.c_contiguous
+    if base.size:
+        hi = int(np.max(base + (trows - 1) * stride + width))
+        assert hi <= min(p.size, g_bits.size, mq.size, vq.size, pb_bits.size)
+        assert int(np.max(sidx)) < min(scale_m.size, scale_v.size)
+    _load().orc_adam8_step_tiles(base.size, _ptr(base), _ptr(trows), _ptr(width), _ptr(stride), _ptr(sidx),
+                                 _ptr(p), _ptr(g_bits), _ptr(mq), _ptr(vq), _ptr(scale_m), _ptr(scale_v),
+                                 _ptr(pb_bits), hp["lr"], hp["beta1"], hp["beta2"], hp["eps"],
+                                 hp["weight_decay"], int(t), float(grad_scale), int(threads))
+
+
 class Bucket:
     """Whole-bucket state on the host, stepped by the oracle.
 
@@ -309,15 +358,22 @@ class Bucket:
     the bf16 copy of padding is set to zero on every step.
     """
 
-    def __init__(self, rows, cols, k, offsets, s, m):
+    def __init__(self, rows, cols, k, offsets, s, m, block_cols=None):
         self.rows, self.cols, self.k = _i64(rows), _i64(cols), _i64(k)
         self.offsets = _i64(offsets)
         self.s, self.m = int(s), int(m)
         self.size = self.s * self.m
-        self.start, self.length = blocks(self.rows, self.cols, self.k, self.offsets)
-        self.sidx = np.arange(self.start.size, dtype=np.int64)
+        bc = np.zeros_like(self.rows) if block_cols is None else _i64(block_cols)
+        self.tiled = bool(np.any((bc > 0) & (bc < self.cols)))
+        if self.tiled:
+            self.tiles = tiles(self.rows, self.cols, self.k, bc, self.offsets)
+            nb = self.tiles[0].size
+        else:
+            self.start, self.length = blocks(self.rows, self.cols, self.k, self.offsets)
+            nb = self.start.size
+        self.sidx = np.arange(nb, dtype=np.int64)
         self.pad = padding_mask(self.rows, self.cols, self.offsets, self.size)
-        S, B = self.size, self.start.size
+        S, B = self.size, nb
         self.p = np.zeros(S, np.float32)
         self.g = np.zeros(S, np.uint16)
         self.mq = np.zeros(S, np.int8)
@@ -331,6 +387,10 @@ class Bucket:
         return slice(o, o + int(self.rows[i] * self.cols[i]))
 
     def step(self, hp, t, grad_scale, threads=1):
-        adam8_step(self.start, self.length, self.sidx, self.p, self.g, self.mq, self.vq,
-                   self.scale_m, self.scale_v, self.pb, hp, t, grad_scale, threads)
+        if self.tiled:
+            adam8_step_tiles(*self.tiles, self.sidx, self.p, self.g, self.mq, self.vq,
+                             self.scale_m, self.scale_v, self.pb, hp, t, grad_scale, threads)
+        else:
+            adam8_step(self.start, self.length, self.sidx, self.p, self.g, self.mq, self.vq,
+                       self.scale_m, self.scale_v, self.pb, hp, t, grad_scale, threads)
         self.pb[self.pad] = 0

@@ -376,6 +376,50 @@ void orc_adam8_step(int64_t n_blocks, const int64_t* start, const int64_t* len, 
     }
 }
 
+// Step a list of 2-D tiles (the 32x32-element blocks of the 8-bit Adam case
+// study: a block of trows[j] rows and width[j] columns of a row-major tensor
+// whose rows are stride[j] elements apart).  Tile j covers the elements
+// base[j] + r * stride[j] + c, r < trows[j], c < width[j], and owns scales
+// scale_m[sidx[j]], scale_v[sidx[j]].  Its elements are gathered in row-major
+// order, stepped as one block by adam8_block, and written back.
+void orc_adam8_step_tiles(int64_t n_tiles, const int64_t* base, const int64_t* trows, const int64_t* width,
+                          const int64_t* stride, const int64_t* sidx, float* p, const uint16_t* g, int8_t* mq,
+                          uint8_t* vq, float* scale_m, float* scale_v, uint16_t* pb, float lr, float beta1,
+                          float beta2, float eps, float wd, int64_t step, float grad_scale, int32_t threads) {
+    const Scalars c = make_scalars(lr, beta1, beta2, eps, wd, step);
+    int64_t maxlen = 0;
+    for (int64_t j = 0; j < n_tiles; ++j) maxlen = std::max(maxlen, trows[j] * width[j]);
+    const size_t L = (size_t)(maxlen > 0 ? maxlen : 1);
+#pragma omp parallel num_threads(threads > 0 ? threads : 1) if (threads > 1)
+    {
+        std::vector<float> mt(L), rt(L), tp(L);
+        std::vector<uint16_t> tg(L), tpb(L);
+        std::vector<int8_t> tm(L);
+        std::vector<uint8_t> tv(L);
+        std::vector<int64_t> at(L);
+#pragma omp for schedule(dynamic, 16)
+        for (int64_t j = 0; j < n_tiles; ++j) {
+            const int64_t n = trows[j] * width[j];
+            for (int64_t r = 0; r < trows[j]; ++r)
+                for (int64_t q = 0; q < width[j]; ++q) at[r * width[j] + q] = base[j] + r * stride[j] + q;
+            for (int64_t i = 0; i < n; ++i) {
+                tp[i] = p[at[i]];
+                tg[i] = g[at[i]];
+                tm[i] = mq[at[i]];
+                tv[i] = vq[at[i]];
+            }
+            adam8_block(n, tp.data(), tg.data(), tm.data(), tv.data(), scale_m + sidx[j], scale_v + sidx[j],
+                        tpb.data(), c, grad_scale, mt.data(), rt.data());
+            for (int64_t i = 0; i < n; ++i) {
+                p[at[i]] = tp[i];
+                mq[at[i]] = tm[i];
+                vq[at[i]] = tv[i];
+                pb[at[i]] = tpb[i];
+            }
+        }
+    }
+}
+
 // The per-step scalars as floats, in the order b1, omb1, b2, omb2, sqrt_bc2,
 // eps_hat, step_hat, decay (for the tests' closed forms).
 void orc_step_scalars(float lr, float beta1, float beta2, float eps, float wd, int64_t t, float* out) {

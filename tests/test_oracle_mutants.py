@@ -61,6 +61,9 @@ MUTANTS = {
     "edge_counts_as_inside": ("    for (int64_t r = o / s + 1; r < m && r * s < o + n; ++r)",
                               "    for (int64_t r = o / s + 1; r < m && r * s <= o + n; ++r)",
                               "test_oracle_layout.py::test_literal_scan_equals_walk"),
+    "tile_transposed": ("                for (int64_t q = 0; q < width[j]; ++q) at[r * width[j] + q] = base[j] + r * stride[j] + q;",
+                        "                for (int64_t q = 0; q < width[j]; ++q) at[r * width[j] + q] = base[j] + q * stride[j] + r;",
+                        "test_oracle_tiles.py::test_golden_tiles_first_step"),
 }
 
 # The same for the oracle's Python part (oracle/__init__.py).
@@ -72,6 +75,11 @@ PY_MUTANTS = {
                                   "test_oracle_rowwise.py::test_golden_rowwise_layout"),
     "rowwise_rank_minor": ("            src = r * C + int(off[t])", "            src = int(off[t]) * m + r",
                            "test_oracle_rowwise.py::test_copy_out_inverts_copy_in"),
+    "tiles_full_last_width": ("                width.append(min(W, C - c0))", "                width.append(W)",
+                              "test_oracle_tiles.py::test_golden_tiles_first_step"),
+    "tiles_rows_as_blocks": ("        W = C if int(bc[i]) <= 0 or int(bc[i]) >= C else int(bc[i])",
+                             "        W = C",
+                             "test_oracle_tiles.py::test_golden_tiles_first_step"),
     "rowwise_unscaled": ("            pack(g[r0 * int(cols[t]):r0 * int(cols[t]) + k], seg, scale)",
                          "            pack(g[r0 * int(cols[t]):r0 * int(cols[t]) + k], seg, 1.0)",
                          "test_oracle_rowwise.py::test_golden_rowwise_layout"),
@@ -93,7 +101,8 @@ def test_pin_catches_planted_mistake(name, tmp_path):
                     ignore=shutil.ignore_patterns("*.so", "__pycache__"))
     shutil.copytree(os.path.join(ROOT, "synth"), work / "synth",
                     ignore=shutil.ignore_patterns("__pycache__"))
-    for f in ("conftest.py", "test_oracle_adam.py", "test_oracle_layout.py", "test_oracle_rowwise.py"):
+    for f in ("conftest.py", "test_oracle_adam.py", "test_oracle_layout.py", "test_oracle_rowwise.py",
+              "test_oracle_tiles.py"):
         shutil.copy(os.path.join(ROOT, "tests", f), work / "tests" / f)
     shutil.copytree(os.path.join(ROOT, "tests", "golden"), work / "tests" / "golden")
     (work / "oracle" / fname).write_text(src.replace(orig, bad))
