@@ -350,6 +350,55 @@ def adam8_step_tiles(base, trows, width, stride, sidx, p, g_bits, mq, vq, scale_
                                  hp["weight_decay"], int(t), float(grad_scale), int(threads))
 
 
+# ------------------------------------------------------------------ Muon ---
+#
+# Distributed Muon on RaggedShard (the pages' case study "8-bit Adam and
+# distributed Muon", paper Sec. 6.3): each 2-D parameter is gathered whole on
+# one rank, its Newton-Schulz preconditioner runs there, and the result goes
+# back to the original placement.  The pages give neither the iteration nor
+# its coefficients; the reading here is Muon as published by its authors
+# (K. Jordan et al., 2024): heavy-ball momentum with the Nesterov form, the
+# quintic Newton-Schulz iteration X <- aX + (b A + c A^2) X with A = X X^T and
+# (a, b, c) = (3.4445, -4.7750, 2.0315), started from the momentum divided by
+# its Frobenius norm, on the wide orientation of the matrix, and an update
+# scaled by sqrt(max(1, rows/cols)) with decoupled weight decay.
+
+NS_COEFFS = (3.4445, -4.7750, 2.0315)
+
+
+def muon_momentum(mom, g_bits, beta, grad_scale, nesterov=True):
+    """Muon's momentum in fp32, every operation rounded on its own, in place
+    on mom (float32):  t = g * grad_scale;  mom = beta * mom + t;  returns the
+    direction U = t + beta * mom (Nesterov) or mom."""
+    assert mom.dtype == np.float32
+    g = (np.asarray(g_bits, dtype=np.uint32) << 16).view(np.float32)
+    b = np.float32(beta)
+    t = g * np.float32(grad_scale)
+    mom[:] = b * mom + t
+    return t + b * mom if nesterov else mom.copy()
+
+
+def newton_schulz(U, steps=5, eps=1e-7):
+    """Orthogonalisation of Muon in float64: X = U / (||U||_F + eps), then
+    `steps` quintic iterations on the orientation with rows <= cols."""
+    X = np.asarray(U, dtype=np.float64)
+    X = X / (np.linalg.norm(X) + eps)
+    tall = X.shape[0] > X.shape[1]
+    if tall:
+        X = X.T
+    a, b, c = NS_COEFFS
+    for _ in range(steps):
+        A = X @ X.T
+        B = b * A + c * (A @ A)
+        X = a * X + B @ X
+    return X.T if tall else X
+
+
+def muon_update_scale(rows, cols):
+    """sqrt(max(1, rows / cols)), the step's shape factor."""
+    return float(np.sqrt(max(1.0, rows / cols)))
+
+
 class Bucket:
     """Whole-bucket state on the host, stepped by the oracle.
 

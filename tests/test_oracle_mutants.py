@@ -80,6 +80,14 @@ PY_MUTANTS = {
     "tiles_rows_as_blocks": ("        W = C if int(bc[i]) <= 0 or int(bc[i]) >= C else int(bc[i])",
                              "        W = C",
                              "test_oracle_tiles.py::test_golden_tiles_first_step"),
+    "ns_swap_bc": ("        B = b * A + c * (A @ A)", "        B = c * A + b * (A @ A)",
+                   "test_oracle_muon.py::test_newton_schulz_is_the_spectral_map"),
+    "ns_no_normalise": ("    X = X / (np.linalg.norm(X) + eps)", "    X = X",
+                        "test_oracle_muon.py::test_newton_schulz_is_the_spectral_map"),
+    "momentum_not_nesterov": ("    return t + b * mom if nesterov else mom.copy()", "    return mom.copy()",
+                              "test_oracle_muon.py::test_momentum_of_a_constant_gradient"),
+    "momentum_unscaled": ("    t = g * np.float32(grad_scale)", "    t = g",
+                          "test_oracle_muon.py::test_momentum_of_a_constant_gradient"),
     "rowwise_unscaled": ("            pack(g[r0 * int(cols[t]):r0 * int(cols[t]) + k], seg, scale)",
                          "            pack(g[r0 * int(cols[t]):r0 * int(cols[t]) + k], seg, 1.0)",
                          "test_oracle_rowwise.py::test_golden_rowwise_layout"),
@@ -102,7 +110,7 @@ def test_pin_catches_planted_mistake(name, tmp_path):
     shutil.copytree(os.path.join(ROOT, "synth"), work / "synth",
                     ignore=shutil.ignore_patterns("__pycache__"))
     for f in ("conftest.py", "test_oracle_adam.py", "test_oracle_layout.py", "test_oracle_rowwise.py",
-              "test_oracle_tiles.py"):
+              "test_oracle_tiles.py", "test_oracle_muon.py"):
         shutil.copy(os.path.join(ROOT, "tests", f), work / "tests" / f)
     shutil.copytree(os.path.join(ROOT, "tests", "golden"), work / "tests" / "golden")
     (work / "oracle" / fname).write_text(src.replace(orig, bad))
