@@ -43,11 +43,22 @@
 extern "C" {
 #endif
 
-/* A tensor of the bucket: row-major rows x cols, quantisation block = k whole
- * rows (the last block may be shorter).  A 1-D tensor of length L is
- * rows=L, cols=1, k=L (one block).  Requires rows, cols, k >= 1, k <= rows. */
+/* A tensor of the bucket: row-major rows x cols.  The layout unit (the
+ * RaggedShard block) is k whole rows, the last one possibly shorter.  A 1-D
+ * tensor of length L is rows=L, cols=1, k=L (one block).
+ *
+ * Quantisation blocks: block_cols = 0 (or >= cols): each k-row block is one
+ * quantisation block.  Otherwise each k-row block is cut into tiles of
+ * block_cols columns, the last one narrower, each with its own scales: the
+ * 2-D blocks (e.g. 32x32 elements, k = block_cols = 32) that the pages' 8-bit
+ * Adam case study allows per parameter (page section "case study: 8-bit Adam
+ * and distributed Muon", paper Sec. 6.3).  Tiles require block_cols a power
+ * of two in [16, 4096] and cols a multiple of 16.
+ *
+ * Requires rows, cols, k >= 1, k <= rows, block_cols >= 0. */
 typedef struct {
     int64_t rows, cols, k;
+    int64_t block_cols;
 } dbuf_tensor_desc;
 
 typedef struct dbuf_plan_s dbuf_plan_t; /* host-only layout, owned by the caller */
@@ -79,8 +90,8 @@ dbuf_status dbuf_plan(const dbuf_tensor_desc* descs, int32_t n, int32_t m, int64
 /* Read a plan.  Any output pointer may be NULL.  offsets[n] (caller-owned)
  * receives each tensor's start in the caller's order.  n_blocks counts the
  * quantisation blocks; blocks are numbered in bucket order (tensors by
- * ascending offset, blocks in row order), which is the index of their
- * scales. */
+ * ascending offset, k-row blocks top to bottom, tiles left to right inside
+ * a k-row block), which is the index of their scales. */
 dbuf_status dbuf_plan_info(const dbuf_plan_t* plan, int64_t* slice_elems, int64_t* bucket_elems,
                            int64_t* padding_elems, int64_t* n_blocks, int64_t* offsets);
 
@@ -222,7 +233,11 @@ dbuf_status dbuf_get_device_status(dbuf_t* db, int32_t* code, void* stream);
  * tools; the kernel's own table holds the same entries).  kind 0: up to 254
  * whole blocks of one tensor, at most 4096 elements counted from the
  * 16-element boundary at or below first_elem; kind 1: one block longer than
- * that, streamed twice; kind 2: a padding range whose bf16 copy is zeroed. */
+ * that, streamed twice; kind 2: a padding range whose bf16 copy is zeroed;
+ * kind 3: columns [c0, c0 + n_elems) of the n_blocks rows of one k-row block
+ * of a tiled tensor (first_elem = row 0, column c0; block_elems = row
+ * stride; reserved = tile width; first_block = scale index of the first
+ * tile), streamed twice. */
 typedef struct {
     int64_t first_elem, first_block, n_elems;
     int32_t block_elems, kind, n_blocks, reserved;

@@ -33,7 +33,8 @@ class DbufError(RuntimeError):
 
 
 class dbuf_tensor_desc(ctypes.Structure):
-    _fields_ = [("rows", ctypes.c_int64), ("cols", ctypes.c_int64), ("k", ctypes.c_int64)]
+    _fields_ = [("rows", ctypes.c_int64), ("cols", ctypes.c_int64), ("k", ctypes.c_int64),
+                ("block_cols", ctypes.c_int64)]
 
 
 class dbuf_adam_hparams(ctypes.Structure):
@@ -125,10 +126,13 @@ class Plan:
             self.handle = None
 
 
-def dbuf_plan(rows, cols, k, m, align_elems=16, max_bucket_elems=0):
+def dbuf_plan(rows, cols, k, m, align_elems=16, max_bucket_elems=0, block_cols=None):
+    """Plan a bucket.  block_cols[i] > 0 (and < cols[i]) cuts tensor i's k-row
+    blocks into tiles of that many columns, each with its own scales."""
     n = len(rows)
-    descs = (dbuf_tensor_desc * max(n, 1))(*[dbuf_tensor_desc(int(r), int(c), int(q))
-                                             for r, c, q in zip(rows, cols, k)])
+    bc = [0] * n if block_cols is None else [int(x) for x in block_cols]
+    descs = (dbuf_tensor_desc * max(n, 1))(*[dbuf_tensor_desc(int(r), int(c), int(q), b)
+                                             for r, c, q, b in zip(rows, cols, k, bc)])
     out = ctypes.c_void_p()
     _check(_lib.dbuf_plan(descs, n, int(m), int(align_elems), int(max_bucket_elems), ctypes.byref(out)))
     return Plan(out.value, n)
@@ -236,7 +240,8 @@ def dbuf_work_table(plan):
     arr = (dbuf_work_item * max(n.value, 1))()
     _check(_lib.dbuf_work_table(plan.handle, arr, n.value, ctypes.byref(n)))
     return [dict(first_elem=a.first_elem, first_block=a.first_block, n_elems=a.n_elems,
-                 block_elems=a.block_elems, kind=a.kind, n_blocks=a.n_blocks) for a in arr[:n.value]]
+                 block_elems=a.block_elems, kind=a.kind, n_blocks=a.n_blocks, tile_cols=a.reserved)
+            for a in arr[:n.value]]
 
 
 def dbuf_clear_device_status(db, stream=None):
@@ -248,7 +253,7 @@ def dbuf_clear_device_status(db, stream=None):
 def dbuf_rowwise_layout(rows, cols, m):
     """Row-wise (FSDP2-style) layout on the host: (chunk_elems, shard_rows, offsets)."""
     n = len(rows)
-    descs = (dbuf_tensor_desc * max(n, 1))(*[dbuf_tensor_desc(int(r), int(c), 1) for r, c in zip(rows, cols)])
+    descs = (dbuf_tensor_desc * max(n, 1))(*[dbuf_tensor_desc(int(r), int(c), 1, 0) for r, c in zip(rows, cols)])
     chunk = ctypes.c_int64()
     q = (ctypes.c_int64 * max(n, 1))()
     off = (ctypes.c_int64 * max(n, 1))()
@@ -263,7 +268,7 @@ class Rowwise:
 
     def __init__(self, rows, cols, m, stream=None):
         n = len(rows)
-        descs = (dbuf_tensor_desc * max(n, 1))(*[dbuf_tensor_desc(int(r), int(c), 1) for r, c in zip(rows, cols)])
+        descs = (dbuf_tensor_desc * max(n, 1))(*[dbuf_tensor_desc(int(r), int(c), 1, 0) for r, c in zip(rows, cols)])
         h = ctypes.c_void_p()
         _check(_lib.dbuf_rowwise_create(descs, n, int(m), _stream(stream), ctypes.byref(h)))
         self.handle, self.n, self.m = h, n, int(m)

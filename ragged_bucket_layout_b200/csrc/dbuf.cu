@@ -54,6 +54,9 @@ void add_zero_tiles(std::vector<Tile>& out, int64_t a, int64_t b) {
         out.push_back(Tile{e, 0, std::min(kZeroChunk, b - e), 0, TILE_ZERO, 0, 0u});
 }
 
+// Elements a LARGE or STRIP entry streams per pass (its sort key).
+int64_t entry_work(const Tile& t) { return t.kind == TILE_STRIP ? t.n * (int64_t)t.nblk : t.n; }
+
 void build_tiles(const dbuf_plan_s& p, std::vector<Tile>& tiles) {
     std::vector<Tile> large, whole, zero;
     int64_t blk = 0, prev_end = 0;
@@ -61,6 +64,19 @@ void build_tiles(const dbuf_plan_s& p, std::vector<Tile>& tiles) {
         const int64_t o = p.offset[id], n = p.rows[id] * p.cols[id], b = p.k[id] * p.cols[id];
         const int64_t nb = cdiv(p.rows[id], p.k[id]);
         if (o > prev_end) add_zero_tiles(zero, prev_end, o);
+        if (!p.tile_cols.empty() && p.tile_cols[id] > 0) {
+            // 2-D blocks: each k-row block in strips of at most kTile columns.
+            const int64_t C = p.cols[id], W = p.tile_cols[id], G = cdiv(C, W);
+            for (int64_t j = 0; j < nb; ++j) {
+                const int64_t r0 = j * p.k[id], nr = std::min(p.k[id], p.rows[id] - r0);
+                for (int64_t c0 = 0; c0 < C; c0 += kTile)
+                    large.push_back(Tile{o + r0 * C + c0, blk + j * G + c0 / W, std::min<int64_t>(kTile, C - c0),
+                                         (int32_t)C, TILE_STRIP, (int32_t)nr, (uint32_t)W});
+            }
+            blk += nb * G;
+            prev_end = o + n;
+            continue;
+        }
         int64_t j = 0;
         while (j < nb) {
             const int64_t e0 = o + j * b;
@@ -83,7 +99,8 @@ void build_tiles(const dbuf_plan_s& p, std::vector<Tile>& tiles) {
     }
     if (prev_end < p.bucket) add_zero_tiles(zero, prev_end, p.bucket);
     // Longest work first so the tail of the grid is short tiles.
-    std::stable_sort(large.begin(), large.end(), [](const Tile& x, const Tile& y) { return x.n > y.n; });
+    std::stable_sort(large.begin(), large.end(),
+                     [](const Tile& x, const Tile& y) { return entry_work(x) > entry_work(y); });
     tiles.clear();
     tiles.reserve(large.size() + whole.size() + zero.size());
     tiles.insert(tiles.end(), large.begin(), large.end());
@@ -151,26 +168,34 @@ struct dbuf_s {
     int norm_grid = 1;  // CTAs of the norm reduction
 };
 
+namespace dbuf_detail {
+int32_t tensors_of(const dbuf_t* db) { return db ? db->plan.n : 0; }
+int device_of(const dbuf_t* db) { return db ? db->device : -1; }
+}  // namespace dbuf_detail
+
 // ----------------------------------------------------------- launches
 
 namespace {
 
 using namespace dbuf_k;
 
-StepC make_step_constants(const dbuf_adam_hparams& hp, float grad_scale) {
+// The step's scalars (double, rounded to float once), each duplicated into
+// a pair for the paired fp32 instructions.
+StepC2 make_step_constants(const dbuf_adam_hparams& hp, float grad_scale) {
     const double B1 = hp.beta1, B2 = hp.beta2, lr = hp.lr, wd = hp.weight_decay, eps = hp.eps;
     const double t = (double)hp.step;
     const double bc1 = 1.0 - std::pow(B1, t);
     const double sq2 = std::sqrt(1.0 - std::pow(B2, t));
-    StepC c;
-    c.b1 = (float)B1;
-    c.omb1 = (float)(1.0 - B1);
-    c.b2 = (float)B2;
-    c.omb2 = (float)(1.0 - B2);
-    c.eps_hat = (float)(eps * sq2);
-    c.step_hat = (float)(lr * sq2 / bc1);
-    c.decay = (float)(1.0 - lr * wd);
-    c.gscale = grad_scale;
+    auto pair = [](double x) { return make_float2((float)x, (float)x); };
+    StepC2 c;
+    c.b1 = pair(B1);
+    c.omb1 = pair(1.0 - B1);
+    c.b2 = pair(B2);
+    c.omb2 = pair(1.0 - B2);
+    c.eps_hat = pair(eps * sq2);
+    c.step_hat = pair(lr * sq2 / bc1);
+    c.decay = pair(1.0 - lr * wd);
+    c.gscale = make_float2(grad_scale, grad_scale);
     return c;
 }
 
@@ -224,7 +249,8 @@ extern "C" dbuf_status dbuf_work_table(const dbuf_plan_t* plan, dbuf_work_item* 
     static_assert(sizeof(dbuf_work_item) == sizeof(Tile), "work item mirrors the device tile");
     const int64_t m = std::min<int64_t>(cap, *n);
     for (int64_t i = 0; i < m; ++i)
-        out[i] = dbuf_work_item{tiles[i].e0, tiles[i].blk0, tiles[i].n, tiles[i].b, tiles[i].kind, tiles[i].nblk, 0};
+        out[i] = dbuf_work_item{tiles[i].e0, tiles[i].blk0, tiles[i].n, tiles[i].b, tiles[i].kind, tiles[i].nblk,
+                                tiles[i].kind == TILE_STRIP ? (int32_t)tiles[i].magic : 0};
     return DBUF_OK;
 }
 
@@ -365,7 +391,7 @@ extern "C" dbuf_status dbuf_adam8_step(dbuf_t* db, const dbuf_adam_hparams* hp, 
     dbuf_status s = step_checks(db, hp, "dbuf_adam8_step");
     if (s != DBUF_OK) return s;
     if (db->h_tiles.empty()) return DBUF_OK;
-    const StepC c = make_step_constants(*hp, grad_scale);
+    const StepC2 c = make_step_constants(*hp, grad_scale);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     adam8_step_kernel<<<(unsigned)db->step_grid, kStepThreads, kStepSmem, st>>>(
         db->tiles, (int64_t)db->h_tiles.size(), db->plan.bucket, db->master, db->param, db->grad, db->mq, db->vq,
@@ -454,7 +480,7 @@ extern "C" dbuf_status dbuf_adam8_step_clipped(dbuf_t* db, const dbuf_adam_hpara
     s = launch_norm(db, grad_scale, max_norm, 1, norm_dev, st, "dbuf_adam8_step_clipped");
     if (s != DBUF_OK) return s;
     if (db->h_tiles.empty()) return DBUF_OK;
-    const StepC c = make_step_constants(*hp, grad_scale);
+    const StepC2 c = make_step_constants(*hp, grad_scale);
     adam8_step_kernel<<<(unsigned)db->step_grid, kStepThreads, kStepSmem, st>>>(
         db->tiles, (int64_t)db->h_tiles.size(), db->plan.bucket, db->master, db->param, db->grad, db->mq, db->vq,
         db->scales, db->plan.n_blocks, c, &db->scratch->gscale_eff, db->status);

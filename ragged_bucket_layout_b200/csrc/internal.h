@@ -13,6 +13,7 @@ struct dbuf_plan_s {
     int64_t align = 16;
     int64_t slice = 0, bucket = 0, padding = 0, n_blocks = 0;
     std::vector<int64_t> rows, cols, k;  // caller order
+    std::vector<int64_t> tile_cols;      // caller order; 0 = whole rows (see dbuf_tensor_desc)
     std::vector<int64_t> offset;         // caller order
     std::vector<int32_t> by_offset;      // tensor ids in bucket order
 };
@@ -22,6 +23,10 @@ namespace dbuf_detail {
 // Thread-local error message of the C-ABI.
 void set_error(const std::string& msg);
 dbuf_status fail(dbuf_status st, const std::string& msg);
+
+// Tensor count and device of a dbuf (for the Muon state in muon.cu).
+int32_t tensors_of(const dbuf_t* db);
+int device_of(const dbuf_t* db);
 
 }  // namespace dbuf_detail
 

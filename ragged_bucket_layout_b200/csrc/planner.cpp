@@ -101,9 +101,15 @@ extern "C" dbuf_status dbuf_plan(const dbuf_tensor_desc* descs, int32_t n, int32
     int64_t total = 0, upper = 0;
     for (int32_t i = 0; i < n; ++i) {
         const dbuf_tensor_desc& d = descs[i];
-        if (d.rows < 1 || d.cols < 1 || d.k < 1 || d.k > d.rows)
+        if (d.rows < 1 || d.cols < 1 || d.k < 1 || d.k > d.rows || d.block_cols < 0)
             return fail(DBUF_EINVAL, "dbuf_plan: tensor " + std::to_string(i) +
-                                         " needs rows, cols, k >= 1 and k <= rows");
+                                         " needs rows, cols, k >= 1, k <= rows and block_cols >= 0");
+        if (d.block_cols > 0 && d.block_cols < d.cols &&
+            (d.block_cols < 16 || d.block_cols > 4096 || (d.block_cols & (d.block_cols - 1)) != 0 || d.cols % 16 != 0))
+            return fail(DBUF_EINVAL, "dbuf_plan: tensor " + std::to_string(i) +
+                                         " tiles need block_cols a power of two in [16, 4096] and cols % 16 == 0");
+        if (d.block_cols > 0 && d.block_cols < d.cols && (d.k > (int64_t(1) << 30) || d.cols > (int64_t(1) << 30)))
+            return fail(DBUF_EINVAL, "dbuf_plan: tensor " + std::to_string(i) + " tiles need k, cols <= 2^30");
         int64_t ne, be;
         if (__builtin_mul_overflow(d.rows, d.cols, &ne) || ne > (int64_t(1) << 46))
             return fail(DBUF_EINVAL, "dbuf_plan: tensor " + std::to_string(i) + " too large");
@@ -172,13 +178,17 @@ extern "C" dbuf_status dbuf_plan(const dbuf_tensor_desc* descs, int32_t n, int32
     p->rows.resize(n);
     p->cols.resize(n);
     p->k.resize(n);
+    p->tile_cols.resize(n);
     p->offset = off;
     int64_t nb = 0;
     for (int32_t i = 0; i < n; ++i) {
         p->rows[i] = descs[i].rows;
         p->cols[i] = descs[i].cols;
         p->k[i] = descs[i].k;
-        nb += cdiv(descs[i].rows, descs[i].k);
+        const int64_t bc = descs[i].block_cols;
+        p->tile_cols[i] = (bc > 0 && bc < descs[i].cols) ? bc : 0;
+        const int64_t per_row_block = p->tile_cols[i] ? cdiv(descs[i].cols, p->tile_cols[i]) : 1;
+        nb += cdiv(descs[i].rows, descs[i].k) * per_row_block;
     }
     p->n_blocks = nb;
     p->by_offset.resize(n);

@@ -161,15 +161,11 @@ struct StepC2 {
     float2 b1, omb1, b2, omb2, eps_hat, step_hat, decay, gscale;
 };
 
-__device__ __forceinline__ StepC2 pairs_of(const StepC& c) {
-    return StepC2{dup(c.b1), dup(c.omb1), dup(c.b2), dup(c.omb2), dup(c.eps_hat), dup(c.step_hat), dup(c.decay),
-                  dup(c.gscale)};
-}
 
 // New m and v for elements (2j, 2j+1) of a vector (sqrt(v) taken per vector).
 __device__ __forceinline__ void new_m_v2(float2 graw, float2 qmf, float2 qvf, float2 dqm, float2 dqv,
-                                         const StepC2& c, float2& m, float2& v) {
-    const float2 g = mul2(graw, c.gscale);
+                                         const StepC2& c, float2 gs, float2& m, float2& v) {
+    const float2 g = mul2(graw, gs);
     const float2 mo = mul2(qmf, dqm);
     const float2 so = mul2(qvf, dqv);
     const float2 vo = mul2(so, so);
@@ -354,7 +350,8 @@ __device__ __forceinline__ void store_codes8(const float* m, const float* r, con
 }
 
 // New m and sqrt(v) of a loaded vector whose elements share dqm/dqv.
-__device__ __forceinline__ void mr8(const In8& x, float dqm, float dqv, const StepC2& c, float* m, float* r) {
+__device__ __forceinline__ void mr8(const In8& x, float dqm, float dqv, const StepC2& c, float2 gs, float* m,
+                                    float* r) {
     const float2 dqm2 = dup(dqm), dqv2 = dup(dqv);
     float2 mm[kV / 2], vv[kV / 2], rr[kV / 2];
 #pragma unroll
@@ -363,7 +360,7 @@ __device__ __forceinline__ void mr8(const In8& x, float dqm, float dqv, const St
         const float2 g = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
         const float2 qmf = ubytes_to_f2(x.mq[j >> 1], 2 * (j & 1), 8388736.0f);
         const float2 qvf = ubytes_to_f2(x.vq[j >> 1], 2 * (j & 1), 8388608.0f);
-        new_m_v2(g, qmf, qvf, dqm2, dqv2, c, mm[j], vv[j]);
+        new_m_v2(g, qmf, qvf, dqm2, dqv2, c, gs, mm[j], vv[j]);
     }
     sqrt_vec(vv, rr);
 #pragma unroll
@@ -382,10 +379,11 @@ __device__ __forceinline__ void mr8(const In8& x, float dqm, float dqv, const St
 // sides (a zero m takes the IEEE path).
 template <bool FULL>
 __device__ __forceinline__ void update8(const unsigned char* st, int li, int lo, int hi, float dqm, float dqv,
-                                        const StepC2& c, const Out& o, float* m, float* r, float& am, float& ar) {
+                                        const StepC2& c, float2 gs, const Out& o, float* m, float* r, float& am,
+                                        float& ar) {
     In8 x;
     load8<FULL>(x, st, li, lo, hi, true);
-    mr8(x, dqm, dqv, c, m, r);
+    mr8(x, dqm, dqv, c, gs, m, r);
     float mn = fabsf(m[0]);
     am = 0.f;
     ar = 0.f;
@@ -462,9 +460,19 @@ __device__ __forceinline__ void block_max_to_smem(int key, float a, float b, Ste
 
 // ------------------------------------------------------------ pipeline
 
+__device__ __forceinline__ bool strip_ok(const Tile& t, int64_t bucket, int64_t n_blocks) {
+    const int64_t C = t.b, W = t.magic;
+    if (C < 16 || (C & 15) || (t.n & 15) || t.n > kTile || t.n > C || t.nblk < 1 || (t.e0 & (kAlign - 1))) return false;
+    if (W < 16 || W > kTile || (W & (W - 1))) return false;
+    if (t.e0 + (int64_t)(t.nblk - 1) * C + t.n > bucket) return false;
+    const int64_t G = (t.n + W - 1) / W;
+    return G <= kMaxStripTiles && t.blk0 >= 0 && t.blk0 + G <= n_blocks;
+}
+
 __device__ __forceinline__ bool tile_ok(const Tile& t, int64_t bucket, int64_t n_blocks) {
     if (t.e0 < 0 || t.n <= 0 || t.e0 + t.n > bucket) return false;
     if (t.kind == TILE_ZERO) return true;
+    if (t.kind == TILE_STRIP) return strip_ok(t, bucket, n_blocks);
     if (t.blk0 < 0 || t.nblk < 1 || t.blk0 + t.nblk > n_blocks) return false;
     if (t.kind == TILE_WHOLE) return t.b > 0 && t.nblk <= kMaxBlk && (t.e0 & (kAlign - 1)) + t.n <= kTile;
     return t.kind == TILE_LARGE && t.nblk == 1;
@@ -473,6 +481,20 @@ __device__ __forceinline__ bool tile_ok(const Tile& t, int64_t bucket, int64_t n
 __device__ __forceinline__ int64_t large_chunks(const Tile& t) {
     const int64_t a0 = t.e0 & ~int64_t(kAlign - 1);
     return (t.e0 + t.n - a0 + kTile - 1) / kTile;
+}
+
+// Chunking of a STRIP entry: rows per chunk, and chunks per pass.
+__device__ __forceinline__ int strip_rows_per_chunk(const Tile& t) { return t.b <= kTile ? kTile / t.b : 1; }
+__device__ __forceinline__ int strip_chunks(const Tile& t) {
+    const int rpc = strip_rows_per_chunk(t);
+    return (t.nblk + rpc - 1) / rpc;
+}
+// First element and length of chunk ch (both multiples of 16).
+__device__ __forceinline__ void strip_chunk(const Tile& t, int ch, int64_t& w0, int& len) {
+    const int rpc = strip_rows_per_chunk(t);
+    const int rows = min(rpc, t.nblk - ch * rpc);
+    w0 = t.e0 + (int64_t)ch * rpc * t.b;
+    len = t.b <= kTile ? rows * t.b : (int)t.n;
 }
 
 // Consumers: wait until stage use k has landed.  Thread 0 waits (bounded),
@@ -503,8 +525,9 @@ __device__ void step_producer(const Tile* __restrict__ tiles, int64_t n_tiles, i
         if (!tile_ok(t, bucket, n_blocks) || t.kind == TILE_ZERO) continue;
         const int64_t a0 = t.e0 & ~int64_t(kAlign - 1);
         const int64_t hi = t.e0 + t.n;
+        const bool strip = t.kind == TILE_STRIP;
         const int passes = t.kind == TILE_WHOLE ? 1 : 2;
-        const int64_t nch = t.kind == TILE_WHOLE ? 1 : large_chunks(t);
+        const int64_t nch = t.kind == TILE_WHOLE ? 1 : strip ? strip_chunks(t) : large_chunks(t);
         for (int pass = 0; pass < passes && !timed_out; ++pass) {
             for (int64_t ch = 0; ch < nch; ++ch) {
                 const uint32_t s = k % kStages;
@@ -513,8 +536,13 @@ __device__ void step_producer(const Tile* __restrict__ tiles, int64_t n_tiles, i
                     break;
                 }
                 unsigned char* st = stages + s * kStageBytes;
-                const int64_t w0 = a0 + ch * kTile;
-                const uint32_t n16 = (uint32_t)((min(hi - w0, (int64_t)kTile) + 15) & ~int64_t(15));
+                int64_t w0 = a0 + ch * kTile;
+                uint32_t n16 = (uint32_t)((min(hi - w0, (int64_t)kTile) + 15) & ~int64_t(15));
+                if (strip) {
+                    int len;
+                    strip_chunk(t, (int)ch, w0, len);
+                    n16 = (uint32_t)len;
+                }
                 uint32_t bytes = n16 * (pass == 0 ? 8u : 4u);
                 int64_t f = 0;
                 uint32_t ns = 0;
@@ -547,8 +575,9 @@ __device__ void step_producer(const Tile* __restrict__ tiles, int64_t n_tiles, i
 // absmax words alternate between two slots by tile parity: the slot of the
 // next single-block tile is cleared here, after every reader of its last use
 // has passed this tile's first barrier.
-__device__ void single_tile(const Tile& t, unsigned char* st, StepShared& sh, uint32_t par, float* master,
-                            uint16_t* param, int8_t* mq, uint8_t* vq, float2* scales, const StepC& c) {
+__device__ void single_tile(const Tile t, unsigned char* st, StepShared& sh, uint32_t par, float* master,
+                            uint16_t* param, int8_t* mq, uint8_t* vq, float2* scales, const StepC2& c2,
+                            float2 gs) {
     const int tid = threadIdx.x;
     const float2 sc = reinterpret_cast<const float2*>(st + kOffS)[t.blk0 & 1];
     const float2 dq = dequant_steps(sc);
@@ -560,7 +589,6 @@ __device__ void single_tile(const Tile& t, unsigned char* st, StepShared& sh, ui
     const int64_t a0 = t.e0 & ~int64_t(kAlign - 1);
     const Out o{master + a0, param + a0, mq + a0, vq + a0};
     const int lo = (int)(t.e0 - a0), hi = lo + (int)t.n;
-    const StepC2 c2 = pairs_of(c);
     float am = 0.f, ar = 0.f;
 #pragma unroll
     for (int j = 0; j < kSub; ++j) {
@@ -568,9 +596,9 @@ __device__ void single_tile(const Tile& t, unsigned char* st, StepShared& sh, ui
         if (!(li < hi && li + kV > lo)) continue;
         float m[kV], r[kV], vm, vr;
         if (li >= lo && li + kV <= hi)
-            update8<true>(st, li, lo, hi, dqm, dqv, c2, o, m, r, vm, vr);
+            update8<true>(st, li, lo, hi, dqm, dqv, c2, gs, o, m, r, vm, vr);
         else
-            update8<false>(st, li, lo, hi, dqm, dqv, c2, o, m, r, vm, vr);
+            update8<false>(st, li, lo, hi, dqm, dqv, c2, gs, o, m, r, vm, vr);
         am = fmaxf(am, vm);
         ar = fmaxf(ar, vr);
         stash_mr(st, li, m, r);
@@ -615,8 +643,8 @@ enum : int { W_MULTI8 = 1, W_MIXED = 2 };
 //   block, found as umulhi(x, magic) = x / b.
 //   W_MIXED: blocks not a multiple of 8 elements, per-element block numbers (rare).
 template <int MODE>
-__device__ void whole_tile(const Tile& t, unsigned char* st, StepShared& sh, float* master, uint16_t* param,
-                           int8_t* mq, uint8_t* vq, float2* scales, const StepC& c) {
+__device__ void whole_tile(const Tile t, unsigned char* st, StepShared& sh, float* master, uint16_t* param,
+                           int8_t* mq, uint8_t* vq, float2* scales, const StepC2& c2, float2 gs) {
     const int tid = threadIdx.x;
     const int nb = t.nblk;
     if (tid < nb) {
@@ -632,7 +660,6 @@ __device__ void whole_tile(const Tile& t, unsigned char* st, StepShared& sh, flo
     const int64_t a0 = t.e0 & ~int64_t(kAlign - 1);
     const Out o{master + a0, param + a0, mq + a0, vq + a0};
     const int lo = (int)(t.e0 - a0), hi = lo + (int)t.n;  // local range of the tile's elements
-    const StepC2 c2 = pairs_of(c);
     const uint32_t b = (uint32_t)t.b, magic = t.magic;
 #pragma unroll
     for (int j = 0; j < kSub; ++j) {
@@ -646,14 +673,15 @@ __device__ void whole_tile(const Tile& t, unsigned char* st, StepShared& sh, flo
             if (any) {
                 key = (int)__umulhi((uint32_t)(max(li, lo) - lo), magic);
                 if (full)
-                    update8<true>(st, li, lo, hi, sh.dqm[key], sh.dqv[key], c2, o, m, r, am, ar);
+                    update8<true>(st, li, lo, hi, sh.dqm[key], sh.dqv[key], c2, gs, o, m, r, am, ar);
                 else
-                    update8<false>(st, li, lo, hi, sh.dqm[key], sh.dqv[key], c2, o, m, r, am, ar);
+                    update8<false>(st, li, lo, hi, sh.dqm[key], sh.dqv[key], c2, gs, o, m, r, am, ar);
                 stash_mr(st, li, m, r);
             }
             block_max_to_smem(key, am, ar, sh);
         } else {
             if (any) {
+                const StepC c{c2.b1.x, c2.omb1.x, c2.b2.x, c2.omb2.x, c2.eps_hat.x, c2.step_hat.x, c2.decay.x, gs.x};
                 In8 x;
                 load8<false>(x, st, li, lo, hi, true);
 #pragma unroll
@@ -716,20 +744,19 @@ __device__ void whole_tile(const Tile& t, unsigned char* st, StepShared& sh, flo
 // A block longer than a tile: pass 1 over its chunks updates the weights and
 // finds the absmax; pass 2 reloads grad and old codes, recomputes m and
 // sqrt(v) and writes the codes.
-__device__ bool large_tile(const Tile& t, uint32_t& k, unsigned char* stages, StepShared& sh, float* master,
-                           uint16_t* param, int8_t* mq, uint8_t* vq, float2* scales, const StepC& c,
-                           int32_t* status) {
+__device__ int64_t large_tile(const Tile t, uint32_t k, unsigned char* stages, StepShared& sh, float* master,
+                           uint16_t* param, int8_t* mq, uint8_t* vq, float2* scales, const StepC2& c2,
+                           float2 gs, int32_t* status) {
     const int tid = threadIdx.x;
     const float2 sc = scales[t.blk0];
     const float2 dq = dequant_steps(sc);
     const float dqm = dq.x, dqv = dq.y;
     const int64_t a0 = t.e0 & ~int64_t(kAlign - 1);
     const int64_t nch = large_chunks(t);
-    const StepC2 c2 = pairs_of(c);
 
     float am = 0.f, ar = 0.f;
     for (int64_t ch = 0; ch < nch; ++ch) {
-        if (!wait_stage(sh, k, status)) return false;
+        if (!wait_stage(sh, k, status)) return -1;
         const unsigned char* st = stages + (k % kStages) * kStageBytes;
         const int64_t w0 = a0 + ch * kTile;
         const Out o{master + w0, param + w0, mq + w0, vq + w0};
@@ -740,9 +767,9 @@ __device__ bool large_tile(const Tile& t, uint32_t& k, unsigned char* stages, St
             if (!(li < hi && li + kV > lo)) continue;
             float m[kV], r[kV], vm, vr;
             if (li >= lo && li + kV <= hi)
-                update8<true>(st, li, lo, hi, dqm, dqv, c2, o, m, r, vm, vr);
+                update8<true>(st, li, lo, hi, dqm, dqv, c2, gs, o, m, r, vm, vr);
             else
-                update8<false>(st, li, lo, hi, dqm, dqv, c2, o, m, r, vm, vr);
+                update8<false>(st, li, lo, hi, dqm, dqv, c2, gs, o, m, r, vm, vr);
             am = fmaxf(am, vm);
             ar = fmaxf(ar, vr);
         }
@@ -776,7 +803,7 @@ __device__ bool large_tile(const Tile& t, uint32_t& k, unsigned char* stages, St
         qv[i] = qv1;
     }
     for (int64_t ch = 0; ch < nch; ++ch) {
-        if (!wait_stage(sh, k, status)) return false;
+        if (!wait_stage(sh, k, status)) return -1;
         const unsigned char* st = stages + (k % kStages) * kStageBytes;
         const int64_t w0 = a0 + ch * kTile;
         const Out o{master + w0, param + w0, mq + w0, vq + w0};
@@ -792,7 +819,7 @@ __device__ bool large_tile(const Tile& t, uint32_t& k, unsigned char* stages, St
                 load8<true>(x, st, li, lo, hi, false);
             else
                 load8<false>(x, st, li, lo, hi, false);
-            mr8(x, dqm, dqv, c2, m, r);
+            mr8(x, dqm, dqv, c2, gs, m, r);
             if (full)
                 store_codes8<true>(m, r, qm, qv, li, lo, hi, o);
             else
@@ -801,10 +828,105 @@ __device__ bool large_tile(const Tile& t, uint32_t& k, unsigned char* stages, St
         release_stage(sh, k);
         ++k;
     }
-    return true;
+    return k;
 }
 
-__device__ void zero_tile(const Tile& t, uint16_t* param) {
+// A STRIP entry (2-D blocks): the columns of a chunk that a thread's vector
+// covers are the same in every chunk (whole rows per chunk, every row start
+// 16-element aligned), so each thread keeps its vectors' tile index, old
+// dequantisation steps and running maxima in registers across the chunks.
+// Pass 1 updates the weights; the tiles' maxima meet in shared memory;
+// pass 2 reloads grad and old codes, recomputes m and sqrt(v) and writes the
+// codes.  Vectors never straddle tiles (tile width and cols are multiples
+// of 16).
+__device__ int64_t strip_tile(const Tile t, uint32_t k, unsigned char* stages, StepShared& sh, float* master,
+                           uint16_t* param, int8_t* mq, uint8_t* vq, float2* scales, const StepC2& c2,
+                           float2 gs, int32_t* status) {
+    const int tid = threadIdx.x;
+    const int C = t.b, W = (int)t.magic;
+    const int G = ((int)t.n + W - 1) / W;
+    const int nch = strip_chunks(t);
+    const int full = C <= kTile ? strip_rows_per_chunk(t) * C : (int)t.n;  // elements of a full chunk
+    int gi[kSub];
+    float2 dq[kSub];
+    float am[kSub], ar[kSub];
+#pragma unroll
+    for (int j = 0; j < kSub; ++j) {
+        const int x = j * (kConsumers * kV) + kV * tid;
+        gi[j] = x < full ? (C <= kTile ? x % C : x) / W : -1;
+        dq[j] = gi[j] >= 0 ? dequant_steps(scales[t.blk0 + gi[j]]) : make_float2(0.f, 0.f);
+        am[j] = 0.f;
+        ar[j] = 0.f;
+    }
+    if (tid < G) {
+        sh.am[tid] = 0u;
+        sh.ar[tid] = 0u;
+    }
+    for (int ch = 0; ch < nch; ++ch) {
+        if (!wait_stage(sh, k, status)) return -1;
+        const unsigned char* st = stages + (k % kStages) * kStageBytes;
+        int64_t w0;
+        int len;
+        strip_chunk(t, ch, w0, len);
+        const Out o{master + w0, param + w0, mq + w0, vq + w0};
+#pragma unroll
+        for (int j = 0; j < kSub; ++j) {
+            const int li = j * (kConsumers * kV) + kV * tid;
+            if (li >= len) continue;
+            float m[kV], r[kV], vm, vr;
+            update8<true>(st, li, 0, len, dq[j].x, dq[j].y, c2, gs, o, m, r, vm, vr);
+            am[j] = fmaxf(am[j], vm);
+            ar[j] = fmaxf(ar[j], vr);
+        }
+        release_stage(sh, k);
+        ++k;
+    }
+#pragma unroll
+    for (int j = 0; j < kSub; ++j) block_max_to_smem(gi[j], am[j], ar[j], sh);
+    named_sync(kBarCons, kConsumers);
+    if (tid < G) {
+        const float AMm = __uint_as_float(sh.am[tid]), AMr = __uint_as_float(sh.ar[tid]);
+        const float2 qf = quant_factors(make_float2(AMm, AMr));
+        sh.qm[tid] = qf.x;
+        sh.qv[tid] = qf.y;
+        scales[t.blk0 + tid] = make_float2(AMm, AMr);
+    }
+    named_sync(kBarCons, kConsumers);
+    float q1[kSub], q2[kSub];
+#pragma unroll
+    for (int j = 0; j < kSub; ++j) {
+        q1[j] = gi[j] >= 0 ? sh.qm[gi[j]] : 0.f;
+        q2[j] = gi[j] >= 0 ? sh.qv[gi[j]] : 0.f;
+    }
+    for (int ch = 0; ch < nch; ++ch) {
+        if (!wait_stage(sh, k, status)) return -1;
+        const unsigned char* st = stages + (k % kStages) * kStageBytes;
+        int64_t w0;
+        int len;
+        strip_chunk(t, ch, w0, len);
+        const Out o{master + w0, param + w0, mq + w0, vq + w0};
+#pragma unroll
+        for (int j = 0; j < kSub; ++j) {
+            const int li = j * (kConsumers * kV) + kV * tid;
+            if (li >= len) continue;
+            In8 x;
+            float m[kV], r[kV], qm[kV], qv[kV];
+            load8<true>(x, st, li, 0, len, false);
+            mr8(x, dq[j].x, dq[j].y, c2, gs, m, r);
+#pragma unroll
+            for (int i = 0; i < kV; ++i) {
+                qm[i] = q1[j];
+                qv[i] = q2[j];
+            }
+            store_codes8<true>(m, r, qm, qv, li, 0, len, o);
+        }
+        release_stage(sh, k);
+        ++k;
+    }
+    return k;
+}
+
+__device__ void zero_tile(const Tile t, uint16_t* param) {
     const int64_t lo = t.e0, hi = t.e0 + t.n;
     const int64_t a0 = t.e0 & ~int64_t(kAlign - 1);
     for (int64_t vb = a0 + 8 * (int64_t)threadIdx.x; vb < hi; vb += 8 * (int64_t)kConsumers) {
@@ -820,14 +942,16 @@ __device__ void zero_tile(const Tile& t, uint16_t* param) {
 __global__ void __launch_bounds__(kStepThreads, DBUF_STEP_MIN_CTAS)
     adam8_step_kernel(const Tile* __restrict__ tiles, int64_t n_tiles, int64_t bucket, float* master,
                       uint16_t* param, const uint16_t* grad, int8_t* mq, uint8_t* vq, float2* scales,
-                      int64_t n_blocks, StepC cp, const float* gscale_dev, int32_t* status) {
+                      int64_t n_blocks, const __grid_constant__ StepC2 cp, const float* gscale_dev,
+                      int32_t* status) {
     extern __shared__ __align__(128) unsigned char stages[];
     __shared__ StepShared sh;
     const int tid = threadIdx.x;
-    // grad_scale comes from device memory when a preceding kernel chose it
-    // (global-norm clipping), so no host round trip is needed.
-    StepC c = cp;
-    if (gscale_dev) c.gscale = *gscale_dev;
+    // The step constants stay in the parameter space (paired operands read
+    // from the constant bank, no registers held).  grad_scale comes from
+    // device memory when a preceding kernel chose it (global-norm clipping),
+    // so no host round trip is needed.
+    const float2 gs = gscale_dev ? dup(*gscale_dev) : cp.gscale;
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sh.full[s], 1);
@@ -843,13 +967,8 @@ __global__ void __launch_bounds__(kStepThreads, DBUF_STEP_MIN_CTAS)
         return;
     }
     uint32_t k = 0, nsingle = 0;
-    // The next table entry is loaded one tile ahead, so its latency hides
-    // behind the current tile.
-    Tile nxt;
-    if ((int64_t)blockIdx.x < n_tiles) nxt = tiles[blockIdx.x];
     for (int64_t ti = blockIdx.x; ti < n_tiles; ti += gridDim.x) {
-        const Tile t = nxt;
-        if (ti + gridDim.x < n_tiles) nxt = tiles[ti + gridDim.x];
+        const Tile t = tiles[ti];
         if (!tile_ok(t, bucket, n_blocks)) {
             if (tid == 0) set_status(status, 2);
             continue;
@@ -860,16 +979,20 @@ __global__ void __launch_bounds__(kStepThreads, DBUF_STEP_MIN_CTAS)
             if (!wait_stage(sh, k, status)) return;
             unsigned char* st = stages + (k % kStages) * kStageBytes;
             if (t.nblk == 1) {
-                single_tile(t, st, sh, nsingle & 1u, master, param, mq, vq, scales, c);
+                single_tile(t, st, sh, nsingle & 1u, master, param, mq, vq, scales, cp, gs);
                 ++nsingle;
             } else if ((t.b & 7) == 0)
-                whole_tile<W_MULTI8>(t, st, sh, master, param, mq, vq, scales, c);
+                whole_tile<W_MULTI8>(t, st, sh, master, param, mq, vq, scales, cp, gs);
             else
-                whole_tile<W_MIXED>(t, st, sh, master, param, mq, vq, scales, c);
+                whole_tile<W_MIXED>(t, st, sh, master, param, mq, vq, scales, cp, gs);
             release_stage(sh, k);
             ++k;
         } else {
-            if (!large_tile(t, k, stages, sh, master, param, mq, vq, scales, c, status)) return;
+            const int64_t nk = t.kind == TILE_STRIP
+                                   ? strip_tile(t, k, stages, sh, master, param, mq, vq, scales, cp, gs, status)
+                                   : large_tile(t, k, stages, sh, master, param, mq, vq, scales, cp, gs, status);
+            if (nk < 0) return;
+            k = (uint32_t)nk;
         }
     }
 }

@@ -27,6 +27,7 @@ class TensorSpec:
     rows: int
     cols: int
     k: int
+    block_cols: int = 0     # > 0: quantisation tiles of k rows x block_cols columns
 
     @property
     def numel(self):
@@ -54,6 +55,10 @@ class Workload:
         c = np.array([t.cols for t in self.tensors], dtype=np.int64)
         k = np.array([t.k for t in self.tensors], dtype=np.int64)
         return r, c, k
+
+    def block_cols(self):
+        """Tile widths (0 = whole rows) as an int64 numpy array in tensor order."""
+        return np.array([t.block_cols for t in self.tensors], dtype=np.int64)
 
 
 def _vec(name, n):
@@ -163,6 +168,35 @@ def ragged_mix(m=4, seed=5):
                     description="ragged mix of block granularities 1..286720 elements")
 
 
+def llama_layer_tiles(m=8):
+    """The Llama layer with 32x32-element quantisation blocks on its matrices
+    (32-row layout granularity), RMSNorm weights as one-row blocks."""
+    ts = [TensorSpec(n, r, c, 32, 32) for n, r, c in LLAMA_SHAPES]
+    ts += [TensorSpec("norm1", 1, 4096, 1), TensorSpec("norm2", 1, 4096, 1)]
+    return Workload(f"llama_layer_32x32_m{m}", ts, m=m, seed=1, steps=10,
+                    description="Llama layer h=4096 with 32x32 blocks on the matrices; m=8")
+
+
+def tiles_mix(m=4, seed=6):
+    """Moderate bucket over every 2-D block path: several rows per chunk
+    (cols <= 4096), one row piece per chunk (cols > 4096) with a narrow last
+    strip, 256 tiles in one strip, a tile as wide as a strip, short last row
+    blocks, and row-block tensors between them."""
+    ts = [
+        TensorSpec("t96", 70, 96, 32, 32),
+        TensorSpec("t4112", 33, 4112, 32, 64),
+        TensorSpec("t1024", 64, 1024, 32, 32),
+        TensorSpec("t4096_16", 5, 4096, 2, 16),
+        TensorSpec("t8192_wide", 40, 8192, 32, 4096),
+        TensorSpec("t48", 48, 48, 16, 16),
+        _vec("bias", 300),
+        TensorSpec("rows100", 20, 100, 3),
+        TensorSpec("t64_k1", 9, 64, 1, 32),
+    ]
+    return Workload(f"tiles_mix_m{m}", ts, m=m, seed=seed, steps=4,
+                    description="2-D block mix: tiles of 16..4096 columns, 1..85 rows per chunk")
+
+
 _BUILDERS = {
     "tiny_m4": lambda: tiny(4),
     "llama_layer_m8": lambda: llama_layer(8),
@@ -175,6 +209,9 @@ _BUILDERS = {
     "copyin_9_m64": lambda: copyin(9, 64),
     "ragged_mix_m4": lambda: ragged_mix(4),
     "ragged_mix_m8": lambda: ragged_mix(8),
+    "tiles_mix_m4": lambda: tiles_mix(4),
+    "tiles_mix_m8": lambda: tiles_mix(8),
+    "llama_layer_32x32_m8": lambda: llama_layer_tiles(8),
 }
 WORKLOAD_NAMES = tuple(_BUILDERS)
 

@@ -38,9 +38,10 @@ class Pair:
     def __init__(self, w, with_oracle=True):
         self.w = w
         self.r, self.c, self.k = w.arrays()
+        self.bc = w.block_cols()
         self.n = self.r * self.c
         self.b = self.k * self.c
-        self.plan = rb.dbuf_plan(self.r, self.c, self.k, w.m, w.align)
+        self.plan = rb.dbuf_plan(self.r, self.c, self.k, w.m, w.align, block_cols=self.bc)
         self.info = rb.dbuf_plan_info(self.plan)
         st, off, s = oracle.plan(self.r, self.c, self.k, w.m, w.align)
         assert st == oracle.OK
@@ -49,7 +50,7 @@ class Pair:
         self.s = s
         self.cum = np.concatenate([[0], np.cumsum(self.n)]).astype(np.int64)
         self.D = rb.DBuffer(self.plan)
-        self.O = oracle.Bucket(self.r, self.c, self.k, off, s, w.m) if with_oracle else None
+        self.O = oracle.Bucket(self.r, self.c, self.k, off, s, w.m, block_cols=self.bc) if with_oracle else None
 
     # ------------------------------------------------------------ inputs
     def load_params(self):

@@ -217,3 +217,58 @@ def test_rowwise_layout_rejects_invalid():
         with pytest.raises(rb.DbufError) as e:
             rb.dbuf_rowwise_layout(rows, cols, m)
         assert e.value.status == rb.DBUF_EINVAL
+
+
+@pytest.mark.parametrize("name", ["tiles_mix_m4", "tiles_mix_m8", "llama_layer_32x32_m8"])
+def test_work_table_tiles_cover_once_and_number_like_oracle(name):
+    """2-D blocks: STRIP entries cover every element of the tiled tensors once
+    (rows x columns with the row stride); the tiles they own are the oracle's
+    tiles in the oracle's numbering; other entries still cover the rest."""
+    w = synth.workload(name)
+    r, c, k = w.arrays()
+    bc = w.block_cols()
+    p = rb.dbuf_plan(r, c, k, w.m, 16, block_cols=bc)
+    info = rb.dbuf_plan_info(p)
+    S = info["bucket"]
+    base, trows, width, stride = oracle.tiles(r, c, k, bc, info["offsets"])
+    assert info["n_blocks"] == base.size
+    cover = np.zeros(S, np.int32)
+    seen = np.zeros(base.size, np.int32)
+    for t in rb.dbuf_work_table(p):
+        e0, n = t["first_elem"], t["n_elems"]
+        if t["kind"] == 3:
+            C, rows, W = t["block_elems"], t["n_blocks"], t["tile_cols"]
+            assert n <= 4096 and n % 16 == 0 and C % 16 == 0 and e0 % 16 == 0
+            for rr in range(rows):
+                cover[e0 + rr * C:e0 + rr * C + n] += 1
+            G = -(-n // W)
+            assert G <= 256
+            for g in range(G):
+                j = t["first_block"] + g
+                assert base[j] == e0 + g * W and trows[j] == rows and stride[j] == C
+                assert width[j] == min(W, n - g * W)
+                seen[j] += 1
+        else:
+            cover[e0:e0 + n] += 1
+            if t["kind"] == 0:
+                seen[t["first_block"]:t["first_block"] + t["n_blocks"]] += 1
+            elif t["kind"] == 1:
+                seen[t["first_block"]] += 1
+    assert np.all(cover == 1)
+    assert np.all(seen == 1)
+
+
+@pytest.mark.parametrize("bc,cols,ok", [(32, 96, True), (16, 4096, True), (4096, 8192, True), (0, 7, True),
+                                        (96, 96, True), (200, 96, True), (24, 96, False), (8, 96, False),
+                                        (32, 100, False), (8192, 16384, False)])
+def test_plan_block_cols_rules(bc, cols, ok):
+    """Tiles need block_cols a power of two in [16, 4096] and cols % 16 == 0;
+    block_cols 0 or >= cols means whole rows and is always accepted."""
+    if ok:
+        p = rb.dbuf_plan([64], [cols], [32], 2, 16, block_cols=[bc])
+        tiles = -(-cols // bc) if 0 < bc < cols else 1
+        assert rb.dbuf_plan_info(p)["n_blocks"] == 2 * tiles
+    else:
+        with pytest.raises(rb.DbufError) as e:
+            rb.dbuf_plan([64], [cols], [32], 2, 16, block_cols=[bc])
+        assert e.value.status == rb.DBUF_EINVAL
