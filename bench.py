@@ -71,6 +71,14 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback 6.65 TB/s"
 
 
+def measured_bf16_peak():
+    """Burst cuBLAS bf16 TFLOP/s from MEASURED_PEAKS.json, else the fallback 1590."""
+    try:
+        return float(json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["bf16_tflops"])
+    except Exception:
+        return 1590.0
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     for f in ("dbuf.cu", "internal.h", "step_kernel.cuh", "fastmath.cuh", "tma.cuh", "tables.h"):
@@ -449,6 +457,35 @@ def run_ours(args):
             "copies_vs_step": (in_ms + out_ms) / (ms_local / args.steps)}
         R.close()
         del sep, flat, outs
+
+        # Distributed Muon on the bucket's matrices (the pages' other case
+        # study): momentum, bf16 Newton-Schulz on the tensor cores (cuBLAS
+        # GEMMs, fp32 accumulation), update; timed per step over all of them.
+        ids = [i for i, t in enumerate(w.tensors) if t.rows >= 2 and t.cols >= 2]
+        if ids:
+            M = rb.Muon(D, ids)
+            hpm = dict(rb.MUON_DEFAULTS)
+            M.step(hpm, gscale)
+            mreps = 5
+            with torch.cuda.stream(stream):
+                m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                m0.record(stream)
+                for _ in range(mreps):
+                    M.step(hpm, gscale)
+                m1.record(stream)
+            m1.synchronize()
+            muon_ms = m0.elapsed_time(m1) / mreps
+            flops = 0
+            for i in ids:
+                sm, lg = min(int(r[i]), int(c[i])), max(int(r[i]), int(c[i]))
+                flops += hpm["ns_steps"] * (4 * sm * sm * lg + 2 * sm ** 3)
+            bf16_peak = measured_bf16_peak()
+            copy_in["muon"] = {"tensors": len(ids), "ns_steps": hpm["ns_steps"], "ms_per_step": muon_ms,
+                               "ns_flops_per_step": flops, "tflops": flops / (muon_ms * 1e-3) / 1e12,
+                               "bf16_peak_tflops": bf16_peak,
+                               "frac_of_bf16_peak": flops / (muon_ms * 1e-3) / 1e12 / bf16_peak,
+                               "gemm": "cuBLAS bf16, fp32 accumulate"}
+            M.close()
 
     peak, peak_src = measured_peak()
     roof = {"bound": "hbm", "achieved": kernel_gbs, "peak": peak, "unit": "GB/s", "frac": kernel_gbs / peak,

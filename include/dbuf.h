@@ -252,6 +252,57 @@ dbuf_status dbuf_clear_device_status(dbuf_t* db, void* stream);
 
 void dbuf_destroy(dbuf_t* db); /* NULL is a no-op; frees only what it allocated */
 
+/* ---------------------------------------------------------- distributed Muon
+ *
+ * Muon on the bucket's 2-D tensors (veScale-FSDP pages, case study "8-bit
+ * Adam and distributed Muon", paper Sec. 6.3: each 2-D parameter is gathered
+ * whole on one rank, Muon's Newton-Schulz preconditioner runs there, and the
+ * result returns to the original placement).  In a bucket every tensor is
+ * whole, so the gather is the tensor's own view; on several GPUs it is a
+ * gather of the tensor's slices to one rank.  The iteration is Muon as its
+ * authors published it (the pages name it without coefficients):
+ *   t = float(grad) * grad_scale;  mom = momentum * mom + t;
+ *   U = t + momentum * mom  (nesterov != 0)  or  U = mom;
+ *   X = U / (||U||_F + eps), then ns_steps times on the orientation with
+ *       rows <= cols:  A = X X^T;  B = b A + c A A;  X = a X + B X,
+ *       (a, b, c) = (3.4445, -4.7750, 2.0315);
+ *   master = master * (1 - lr * weight_decay) - lr * sqrt(max(1, rows/cols)) * X;
+ *   param = bf16(master).
+ * Momentum and its norm are fp32 with fp64 sums (deterministic); the
+ * iteration is bf16 with fp32 accumulation, its matrix products cuBLAS GEMMs
+ * on the tensor cores. */
+typedef struct dbuf_muon_s dbuf_muon_t;
+
+typedef struct {
+    float lr, momentum, weight_decay, eps;
+    int32_t ns_steps; /* >= 1 */
+    int32_t nesterov;
+} dbuf_muon_hparams;
+
+/* Muon state for the tensors ids[n] (indices in the plan's caller order;
+ * each with rows, cols >= 2) of db: fp32 momentum per tensor (zeroed on
+ * `stream`), bf16 workspaces sized for the largest tensor, a cuBLAS handle.
+ * One cudaMalloc besides cuBLAS's own; the call waits for the zeroing.  db
+ * must outlive the state.  DBUF_EINVAL for a bad or repeated id. */
+dbuf_status dbuf_muon_create(dbuf_t* db, const int32_t* ids, int32_t n, void* stream, dbuf_muon_t** out);
+
+/* One Muon step of every listed tensor, in list order, on `stream`: reads
+ * the bucket's bf16 grads, updates the momentum, fp32 master weights and
+ * bf16 params in place.  The state is bound to db's device; calls on one
+ * state must not overlap. */
+dbuf_status dbuf_muon_step(dbuf_muon_t* mu, const dbuf_muon_hparams* hp, float grad_scale, void* stream);
+
+/* The orthogonalisation alone: x_bf16 = NS_steps(u / (||u||_F + eps)) for a
+ * row-major fp32 rows x cols matrix u (device pointers; rows*cols and
+ * min(rows, cols)^2 within the state's workspace, else DBUF_EINVAL). */
+dbuf_status dbuf_muon_orthogonalize(dbuf_muon_t* mu, const float* u, int64_t rows, int64_t cols, int32_t ns_steps,
+                                    float eps, void* x_bf16, void* stream);
+
+/* Device pointer and length of listed tensor i's momentum (row-major fp32). */
+dbuf_status dbuf_muon_momentum(const dbuf_muon_t* mu, int32_t i, float** ptr, int64_t* n);
+
+void dbuf_muon_destroy(dbuf_muon_t* mu); /* NULL is a no-op */
+
 /* ------------------------------------------------ row-wise baseline layout
  *
  * The layout RaggedShard replaces, for measuring what it saves: row-wise even

@@ -77,6 +77,11 @@ _SIGS = {
     "dbuf_work_table": (ctypes.c_int, [_P, ctypes.POINTER(dbuf_work_item), _i64, _pi64]),
     "dbuf_destroy": (None, [_P]),
     "dbuf_last_error": (ctypes.c_char_p, []),
+    "dbuf_muon_create": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int32), _i32, _P, _PP]),
+    "dbuf_muon_step": (ctypes.c_int, [_P, _P, _f32, _P]),
+    "dbuf_muon_orthogonalize": (ctypes.c_int, [_P, _P, _i64, _i64, _i32, _f32, _P, _P]),
+    "dbuf_muon_momentum": (ctypes.c_int, [_P, _i32, ctypes.POINTER(ctypes.POINTER(ctypes.c_float)), _pi64]),
+    "dbuf_muon_destroy": (None, [_P]),
     "dbuf_rowwise_layout": (ctypes.c_int, [ctypes.POINTER(dbuf_tensor_desc), _i32, _i32, _pi64, _pi64, _pi64]),
     "dbuf_rowwise_create": (ctypes.c_int, [ctypes.POINTER(dbuf_tensor_desc), _i32, _i32, _P, _PP]),
     "dbuf_rowwise_info": (ctypes.c_int, [_P, _pi64, _pi64, _pi64]),
@@ -246,6 +251,70 @@ def dbuf_work_table(plan):
 
 def dbuf_clear_device_status(db, stream=None):
     _check(_lib.dbuf_clear_device_status(db, _stream(stream)))
+
+
+# ------------------------------------------------------ distributed Muon
+
+class dbuf_muon_hparams(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("momentum", ctypes.c_float), ("weight_decay", ctypes.c_float),
+                ("eps", ctypes.c_float), ("ns_steps", ctypes.c_int32), ("nesterov", ctypes.c_int32)]
+
+
+MUON_DEFAULTS = dict(lr=0.02, momentum=0.95, weight_decay=0.0, eps=1e-7, ns_steps=5, nesterov=1)
+
+
+class Muon:
+    """Muon state for some 2-D tensors of a DBuffer (owner of a dbuf_muon_t);
+    all work goes through the C-ABI on the DBuffer's stream."""
+
+    def __init__(self, dbuffer, ids):
+        self.D = dbuffer
+        ids = [int(i) for i in ids]
+        arr = (ctypes.c_int32 * max(len(ids), 1))(*ids)
+        h = ctypes.c_void_p()
+        _check(_lib.dbuf_muon_create(dbuffer.handle, arr, len(ids), _stream(dbuffer.stream), ctypes.byref(h)))
+        self.handle, self.ids = h, ids
+        self._destroy = _lib.dbuf_muon_destroy   # held here: module globals may be gone at interpreter exit
+
+    def close(self):
+        if getattr(self, "handle", None):
+            self._destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        self.close()
+
+    def step(self, hp, grad_scale):
+        h = dbuf_muon_hparams(**{**MUON_DEFAULTS, **hp})
+        _check(_lib.dbuf_muon_step(self.handle, ctypes.byref(h), float(grad_scale), _stream(self.D.stream)))
+
+    def orthogonalize(self, u, steps=5, eps=1e-7, out=None):
+        """bf16 Newton-Schulz of a 2-D fp32 CUDA tensor."""
+        import torch
+        rows, cols = u.shape
+        out = torch.empty((rows, cols), dtype=torch.bfloat16, device=u.device) if out is None else out
+        _check(_lib.dbuf_muon_orthogonalize(self.handle, u.data_ptr(), rows, cols, int(steps), float(eps),
+                                            out.data_ptr(), _stream(self.D.stream)))
+        return out
+
+    def momentum(self, j):
+        """fp32 momentum of listed tensor j as a 1-D view (borrowed device memory)."""
+        import torch
+        p, n = ctypes.POINTER(ctypes.c_float)(), ctypes.c_int64()
+        _check(_lib.dbuf_muon_momentum(self.handle, int(j), ctypes.byref(p), ctypes.byref(n)))
+        addr = ctypes.cast(p, ctypes.c_void_p).value
+        return _wrap_device_f32(addr, n.value, self.D.base)
+
+
+def _wrap_device_f32(addr, n, like):
+    """A float32 tensor over n elements of device memory at addr (no copy)."""
+    import torch
+
+    class _Arr:
+        pass
+    a = _Arr()
+    a.__cuda_array_interface__ = {"shape": (n,), "typestr": "<f4", "data": (addr, False), "version": 3}
+    return torch.as_tensor(a, device=like.device)
 
 
 # --------------------------------------------- row-wise baseline layout

@@ -7,7 +7,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libdbuf.so")
-SOURCES = [os.path.join(CSRC, f) for f in ("dbuf.cu", "rowwise.cu", "planner.cpp")]
+SOURCES = [os.path.join(CSRC, f) for f in ("dbuf.cu", "rowwise.cu", "muon.cu", "planner.cpp")]
 HEADERS = [os.path.join(CSRC, f) for f in sorted(os.listdir(CSRC)) if f.endswith((".h", ".cuh"))] + [
     os.path.join(ROOT, "include", "dbuf.h")]
 
@@ -40,7 +40,7 @@ def build(force=False, verbose=False):
     """Compile csrc/*.cu|cpp into ragged_bucket_layout_b200/libdbuf.so."""
     if not force and not stale():
         return LIB
-    cmd = [nvcc(), *NVCC_FLAGS, *(["-Xptxas", "-v"] if verbose else []), "-o", LIB, *SOURCES, "-lcudart"]
+    cmd = [nvcc(), *NVCC_FLAGS, *(["-Xptxas", "-v"] if verbose else []), "-o", LIB, *SOURCES, "-lcudart", "-lcublas"]
     subprocess.check_call(cmd)
     return LIB
 
