@@ -105,8 +105,10 @@ def test_pin_catches_planted_mistake(name, tmp_path):
     assert src.count(orig) == 1, f"mutation site of {name} not found once"
     work = tmp_path / "repo"
     os.makedirs(work / "tests")
-    shutil.copytree(os.path.join(ROOT, "oracle"), work / "oracle",
-                    ignore=shutil.ignore_patterns("*.so", "__pycache__"))
+    # A mistake planted in the Python part keeps the built library (same
+    # source); one in oracle.cpp is rebuilt from the edited copy.
+    skip = ("__pycache__",) if fname != "oracle.cpp" else ("*.so", "__pycache__")
+    shutil.copytree(os.path.join(ROOT, "oracle"), work / "oracle", ignore=shutil.ignore_patterns(*skip))
     shutil.copytree(os.path.join(ROOT, "synth"), work / "synth",
                     ignore=shutil.ignore_patterns("__pycache__"))
     for f in ("conftest.py", "test_oracle_adam.py", "test_oracle_layout.py", "test_oracle_rowwise.py",
