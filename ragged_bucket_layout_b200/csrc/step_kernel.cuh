@@ -520,6 +520,7 @@ __device__ void step_producer(const Tile* __restrict__ tiles, int64_t n_tiles, i
                               const float2* scales, unsigned char* stages, StepShared& sh, int32_t* status) {
     uint32_t k = 0;
     bool timed_out = false;
+    const uint64_t keep = l2_policy_evict_last(), drop = l2_policy_evict_first();
     for (int64_t ti = blockIdx.x; ti < n_tiles && !timed_out; ti += gridDim.x) {
         const Tile t = tiles[ti];
         if (!tile_ok(t, bucket, n_blocks) || t.kind == TILE_ZERO) continue;
@@ -552,10 +553,20 @@ __device__ void step_producer(const Tile* __restrict__ tiles, int64_t n_tiles, i
                     bytes += ns * 8u;
                 }
                 mbar_arrive_expect_tx(&sh.full[s], bytes);
-                bulk_g2s(st + kOffG, grad + w0, n16 * 2u, &sh.full[s]);
-                if (pass == 0) bulk_g2s(st + kOffP, master + w0, n16 * 4u, &sh.full[s]);
-                bulk_g2s(st + kOffMQ, mq + w0, n16, &sh.full[s]);
-                bulk_g2s(st + kOffVQ, vq + w0, n16, &sh.full[s]);
+                if (passes == 1) {
+                    bulk_g2s(st + kOffG, grad + w0, n16 * 2u, &sh.full[s]);
+                    bulk_g2s(st + kOffP, master + w0, n16 * 4u, &sh.full[s]);
+                    bulk_g2s(st + kOffMQ, mq + w0, n16, &sh.full[s]);
+                    bulk_g2s(st + kOffVQ, vq + w0, n16, &sh.full[s]);
+                } else {
+                    // Two-pass entries read grad and codes again in pass 2:
+                    // ask L2 to keep them until then, and to drop them after.
+                    const uint64_t pol = pass == 0 ? keep : drop;
+                    bulk_g2s_hint(st + kOffG, grad + w0, n16 * 2u, &sh.full[s], pol);
+                    if (pass == 0) bulk_g2s_hint(st + kOffP, master + w0, n16 * 4u, &sh.full[s], drop);
+                    bulk_g2s_hint(st + kOffMQ, mq + w0, n16, &sh.full[s], pol);
+                    bulk_g2s_hint(st + kOffVQ, vq + w0, n16, &sh.full[s], pol);
+                }
                 if (ns) bulk_g2s(st + kOffS, scales + f, ns * 8u, &sh.full[s]);
                 ++k;
             }
