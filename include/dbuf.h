@@ -191,9 +191,18 @@ dbuf_status dbuf_adam8_step_clipped(dbuf_t* db, const dbuf_adam_hparams* hp, flo
 
 /* The same step with host buffers at both ends (the end-to-end path): copies
  * grads_host (bucket_elems bf16, caller's host memory, pinned for overlap)
- * into the grad bucket, runs dbuf_adam8_step, and copies the bf16 param
- * bucket back to params_bf16_host (bucket_elems bf16).  All three are
- * enqueued on `stream`; the caller synchronises before reading the output. */
+ * into the grad bucket, runs the step, and copies the bf16 param bucket back
+ * to params_bf16_host (bucket_elems bf16).  On buckets of more than 4M
+ * elements this is a pipeline over up to 16 chunks of the bucket:
+ *   - a chunk's gradients come in on a copy stream of the dbuf's own;
+ *   - the chunk is stepped on `stream` once they have landed;
+ *   - its params go out on a second internal stream while later chunks
+ *     are still coming in;
+ * so the two copy directions and the step overlap.  The results equal
+ * dbuf_adam8_step's bit for bit.  Everything is ordered after the work
+ * already queued on `stream`, and work queued on `stream` afterwards runs
+ * after the last copy out.  The caller synchronises `stream` before reading
+ * the output. */
 dbuf_status dbuf_adam8_step_host(dbuf_t* db, const dbuf_adam_hparams* hp, float grad_scale,
                                  const void* grads_host, void* params_bf16_host, void* stream);
 

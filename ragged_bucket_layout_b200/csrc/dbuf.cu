@@ -49,29 +49,46 @@ using namespace dbuf_k;
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-void add_zero_tiles(std::vector<Tile>& out, int64_t a, int64_t b) {
-    for (int64_t e = a; e < b; e += kZeroChunk)
-        out.push_back(Tile{e, 0, std::min(kZeroChunk, b - e), 0, TILE_ZERO, 0, 0u});
+// Entries in bucket order with the element range each one reads and writes
+// (a STRIP: its whole k-row block), for the chunked host-buffer step.
+struct PosTiles {
+    std::vector<Tile> tiles;
+    std::vector<int64_t> lo, hi;
+    void add(const Tile& t, int64_t a, int64_t b) {
+        tiles.push_back(t);
+        lo.push_back(a);
+        hi.push_back(b);
+    }
+};
+
+void add_zero_tiles(std::vector<Tile>& out, PosTiles* pos, int64_t a, int64_t b) {
+    for (int64_t e = a; e < b; e += kZeroChunk) {
+        const Tile t{e, 0, std::min(kZeroChunk, b - e), 0, TILE_ZERO, 0, 0u};
+        out.push_back(t);
+        if (pos) pos->add(t, t.e0, t.e0 + t.n);
+    }
 }
 
 // Elements a LARGE or STRIP entry streams per pass (its sort key).
 int64_t entry_work(const Tile& t) { return t.kind == TILE_STRIP ? t.n * (int64_t)t.nblk : t.n; }
 
-void build_tiles(const dbuf_plan_s& p, std::vector<Tile>& tiles) {
+void build_tiles(const dbuf_plan_s& p, std::vector<Tile>& tiles, PosTiles* pos = nullptr) {
     std::vector<Tile> large, whole, zero;
     int64_t blk = 0, prev_end = 0;
     for (int32_t id : p.by_offset) {
         const int64_t o = p.offset[id], n = p.rows[id] * p.cols[id], b = p.k[id] * p.cols[id];
         const int64_t nb = cdiv(p.rows[id], p.k[id]);
-        if (o > prev_end) add_zero_tiles(zero, prev_end, o);
+        if (o > prev_end) add_zero_tiles(zero, pos, prev_end, o);
         if (!p.tile_cols.empty() && p.tile_cols[id] > 0) {
             // 2-D blocks: each k-row block in strips of at most kTile columns.
             const int64_t C = p.cols[id], W = p.tile_cols[id], G = cdiv(C, W);
             for (int64_t j = 0; j < nb; ++j) {
                 const int64_t r0 = j * p.k[id], nr = std::min(p.k[id], p.rows[id] - r0);
-                for (int64_t c0 = 0; c0 < C; c0 += kTile)
+                for (int64_t c0 = 0; c0 < C; c0 += kTile) {
                     large.push_back(Tile{o + r0 * C + c0, blk + j * G + c0 / W, std::min<int64_t>(kTile, C - c0),
                                          (int32_t)C, TILE_STRIP, (int32_t)nr, (uint32_t)W});
+                    if (pos) pos->add(large.back(), o + r0 * C, o + (r0 + nr) * C);
+                }
             }
             blk += nb * G;
             prev_end = o + n;
@@ -87,17 +104,19 @@ void build_tiles(const dbuf_plan_s& p, std::vector<Tile>& tiles) {
                     const uint32_t magic = b >= 2 ? (uint32_t)(((uint64_t(1) << 32) + (uint64_t)b - 1) / (uint64_t)b) : 0u;
                     whole.push_back(Tile{e0, blk + j, std::min(q * b, n - j * b), (int32_t)b, TILE_WHOLE,
                                          (int32_t)q, magic});
+                    if (pos) pos->add(whole.back(), e0, e0 + whole.back().n);
                     j += q;
                     continue;
                 }
             }
             large.push_back(Tile{e0, blk + j, std::min(b, n - j * b), 0, TILE_LARGE, 1, 0u});
+            if (pos) pos->add(large.back(), e0, e0 + large.back().n);
             j += 1;
         }
         blk += nb;
         prev_end = o + n;
     }
-    if (prev_end < p.bucket) add_zero_tiles(zero, prev_end, p.bucket);
+    if (prev_end < p.bucket) add_zero_tiles(zero, pos, prev_end, p.bucket);
     // Longest work first so the tail of the grid is short tiles.
     std::stable_sort(large.begin(), large.end(),
                      [](const Tile& x, const Tile& y) { return entry_work(x) > entry_work(y); });
@@ -120,8 +139,30 @@ void build_pack_chunks(const dbuf_plan_s& p, std::vector<PackChunk>& chunks, std
     first[p.n] = (int64_t)chunks.size();
 }
 
+// Consecutive runs of the bucket-order entries, each covering a contiguous
+// element range [lo, hi) of about `target` elements; the ranges partition
+// the bucket.  A run never ends inside a k-row block's strips.
+struct HostChunk {
+    int64_t t0, t1, lo, hi;
+};
+
+void build_host_chunks(const PosTiles& pos, int64_t target, std::vector<HostChunk>& out) {
+    out.clear();
+    const int64_t n = (int64_t)pos.tiles.size();
+    int64_t t0 = 0;
+    while (t0 < n) {
+        int64_t t1 = t0, hi = pos.hi[t0];
+        while (t1 < n && (pos.lo[t1] < hi || hi - pos.lo[t0] < target)) {
+            hi = std::max(hi, pos.hi[t1]);
+            ++t1;
+        }
+        out.push_back(HostChunk{t0, t1, pos.lo[t0], hi});
+        t0 = t1;
+    }
+}
+
 struct Layout {
-    size_t master, param, grad, mq, vq, scales, tiles, chunks, status, scratch, total;
+    size_t master, param, grad, mq, vq, scales, tiles, pos_tiles, chunks, status, scratch, total;
 };
 
 Layout layout_of(const dbuf_plan_s& p, size_t n_tiles, size_t n_chunks) {
@@ -135,6 +176,7 @@ Layout layout_of(const dbuf_plan_s& p, size_t n_tiles, size_t n_chunks) {
     L.vq = at;     at = align256(at + S);
     L.scales = at; at = align256(at + ((size_t)p.n_blocks + 2) * 8);
     L.tiles = at;  at = align256(at + n_tiles * sizeof(Tile));
+    L.pos_tiles = at; at = align256(at + n_tiles * sizeof(Tile));
     L.chunks = at; at = align256(at + n_chunks * sizeof(PackChunk));
     L.status = at; at = align256(at + 16);
     L.scratch = at; at = align256(at + sizeof(NormScratch));
@@ -158,15 +200,32 @@ struct dbuf_s {
     uint8_t* vq = nullptr;
     float2* scales = nullptr;
     Tile* tiles = nullptr;
+    Tile* pos_tiles = nullptr;   // the same entries in bucket order (host-buffer step)
     PackChunk* chunks = nullptr;
     int32_t* status = nullptr;
     NormScratch* scratch = nullptr;
     std::vector<Tile> h_tiles;
+    PosTiles h_pos;
+    std::vector<HostChunk> h_host_chunks;
+    // Pipeline of the host-buffer step: copies in and out on their own
+    // streams, overlapping the step of other chunks.
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    cudaEvent_t ev_start = nullptr, ev_done = nullptr;
+    std::vector<cudaEvent_t> ev_in, ev_step;
     std::vector<PackChunk> h_chunks;
     std::vector<int64_t> h_chunk_first;
     int step_grid = 0;  // persistent CTAs of the step kernel
     int norm_grid = 1;  // CTAs of the norm reduction
 };
+
+static void release_pipeline(dbuf_s* db) {
+    for (cudaEvent_t e : db->ev_in) if (e) cudaEventDestroy(e);
+    for (cudaEvent_t e : db->ev_step) if (e) cudaEventDestroy(e);
+    if (db->ev_start) cudaEventDestroy(db->ev_start);
+    if (db->ev_done) cudaEventDestroy(db->ev_done);
+    if (db->s_in) cudaStreamDestroy(db->s_in);
+    if (db->s_out) cudaStreamDestroy(db->s_out);
+}
 
 namespace dbuf_detail {
 int32_t tensors_of(const dbuf_t* db) { return db ? db->plan.n : 0; }
@@ -264,7 +323,10 @@ extern "C" dbuf_status dbuf_create(const dbuf_plan_t* plan, void* device_base, s
     dbuf_s* db = new (std::nothrow) dbuf_s;
     if (!db) return fail(DBUF_ENOMEM, "dbuf_create: out of host memory");
     db->plan = *plan;
-    build_tiles(db->plan, db->h_tiles);
+    build_tiles(db->plan, db->h_tiles, &db->h_pos);
+    // Chunks of the host-buffer pipeline: at most 16, at least 4M elements each.
+    build_host_chunks(db->h_pos, std::max<int64_t>(int64_t(1) << 22, cdiv(db->plan.bucket, 16)),
+                      db->h_host_chunks);
     build_pack_chunks(db->plan, db->h_chunks, db->h_chunk_first);
     db->lay = layout_of(db->plan, db->h_tiles.size(), db->h_chunks.size());
     db->bytes = db->lay.total;
@@ -315,6 +377,7 @@ extern "C" dbuf_status dbuf_create(const dbuf_plan_t* plan, void* device_base, s
     db->vq = reinterpret_cast<uint8_t*>(b + db->lay.vq);
     db->scales = reinterpret_cast<float2*>(b + db->lay.scales);
     db->tiles = reinterpret_cast<Tile*>(b + db->lay.tiles);
+    db->pos_tiles = reinterpret_cast<Tile*>(b + db->lay.pos_tiles);
     db->chunks = reinterpret_cast<PackChunk*>(b + db->lay.chunks);
     db->status = reinterpret_cast<int32_t*>(b + db->lay.status);
     db->scratch = reinterpret_cast<NormScratch*>(b + db->lay.scratch);
@@ -322,10 +385,26 @@ extern "C" dbuf_status dbuf_create(const dbuf_plan_t* plan, void* device_base, s
     if (e == cudaSuccess && !db->h_tiles.empty())
         e = cudaMemcpyAsync(db->tiles, db->h_tiles.data(), db->h_tiles.size() * sizeof(Tile),
                             cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess && !db->h_pos.tiles.empty())
+        e = cudaMemcpyAsync(db->pos_tiles, db->h_pos.tiles.data(), db->h_pos.tiles.size() * sizeof(Tile),
+                            cudaMemcpyHostToDevice, st);
     if (e == cudaSuccess && !db->h_chunks.empty())
         e = cudaMemcpyAsync(db->chunks, db->h_chunks.data(), db->h_chunks.size() * sizeof(PackChunk),
                             cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess && db->h_host_chunks.size() > 1) {
+        e = cudaStreamCreateWithFlags(&db->s_in, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&db->s_out, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&db->ev_start, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&db->ev_done, cudaEventDisableTiming);
+        db->ev_in.assign(db->h_host_chunks.size(), nullptr);
+        db->ev_step.assign(db->h_host_chunks.size(), nullptr);
+        for (size_t i = 0; e == cudaSuccess && i < db->h_host_chunks.size(); ++i) {
+            e = cudaEventCreateWithFlags(&db->ev_in[i], cudaEventDisableTiming);
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&db->ev_step[i], cudaEventDisableTiming);
+        }
+    }
     if (e != cudaSuccess) {
+        release_pipeline(db);
         if (db->owns) cudaFree(db->base);
         delete db;
         return fail(DBUF_ECUDA, std::string("dbuf_create: initialising the bucket: ") + cudaGetErrorString(e));
@@ -336,6 +415,7 @@ extern "C" dbuf_status dbuf_create(const dbuf_plan_t* plan, void* device_base, s
 
 extern "C" void dbuf_destroy(dbuf_t* db) {
     if (!db) return;
+    release_pipeline(db);
     if (db->owns && db->base) cudaFree(db->base);
     delete db;
 }
@@ -496,12 +576,48 @@ extern "C" dbuf_status dbuf_adam8_step_host(dbuf_t* db, const dbuf_adam_hparams*
         return fail(DBUF_EINVAL, "dbuf_adam8_step_host: host buffer is NULL");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const size_t bytes = (size_t)db->plan.bucket * 2;
-    if (bytes) CUDA_TRY(cudaMemcpyAsync(db->grad, grads_host, bytes, cudaMemcpyHostToDevice, st),
-                        "dbuf_adam8_step_host: copy in");
-    s = dbuf_adam8_step(db, hp, grad_scale, stream);
-    if (s != DBUF_OK) return s;
-    if (bytes) CUDA_TRY(cudaMemcpyAsync(params_bf16_host, db->param, bytes, cudaMemcpyDeviceToHost, st),
-                        "dbuf_adam8_step_host: copy out");
+    if (db->h_host_chunks.size() <= 1) {
+        if (bytes) CUDA_TRY(cudaMemcpyAsync(db->grad, grads_host, bytes, cudaMemcpyHostToDevice, st),
+                            "dbuf_adam8_step_host: copy in");
+        s = dbuf_adam8_step(db, hp, grad_scale, stream);
+        if (s != DBUF_OK) return s;
+        if (bytes) CUDA_TRY(cudaMemcpyAsync(params_bf16_host, db->param, bytes, cudaMemcpyDeviceToHost, st),
+                            "dbuf_adam8_step_host: copy out");
+        return DBUF_OK;
+    }
+    // Chunked pipeline: chunk i's gradients arrive on s_in, its entries are
+    // stepped on `stream` once they have, and its bf16 params leave on s_out
+    // once stepped, so the two copy directions and the step overlap.  The
+    // chunks' element ranges partition the bucket and every entry reads and
+    // writes inside its chunk's range (a bulk copy may also read up to 15
+    // elements beyond it, into lanes the step ignores).
+    const StepC2 c = make_step_constants(*hp, grad_scale);
+    const char* gh = static_cast<const char*>(grads_host);
+    char* ph = static_cast<char*>(params_bf16_host);
+    CUDA_TRY(cudaEventRecord(db->ev_start, st), "dbuf_adam8_step_host: record");
+    CUDA_TRY(cudaStreamWaitEvent(db->s_in, db->ev_start, 0), "dbuf_adam8_step_host: wait");
+    CUDA_TRY(cudaStreamWaitEvent(db->s_out, db->ev_start, 0), "dbuf_adam8_step_host: wait");
+    for (size_t i = 0; i < db->h_host_chunks.size(); ++i) {
+        const HostChunk& hc = db->h_host_chunks[i];
+        const size_t off = (size_t)hc.lo * 2, len = (size_t)(hc.hi - hc.lo) * 2;
+        CUDA_TRY(cudaMemcpyAsync(reinterpret_cast<char*>(db->grad) + off, gh + off, len, cudaMemcpyHostToDevice,
+                                 db->s_in),
+                 "dbuf_adam8_step_host: copy in");
+        CUDA_TRY(cudaEventRecord(db->ev_in[i], db->s_in), "dbuf_adam8_step_host: record");
+        CUDA_TRY(cudaStreamWaitEvent(st, db->ev_in[i], 0), "dbuf_adam8_step_host: wait");
+        const int64_t nt = hc.t1 - hc.t0;
+        adam8_step_kernel<<<(unsigned)std::min<int64_t>(nt, db->step_grid), kStepThreads, kStepSmem, st>>>(
+            db->pos_tiles + hc.t0, nt, db->plan.bucket, db->master, db->param, db->grad, db->mq, db->vq,
+            db->scales, db->plan.n_blocks, c, nullptr, db->status);
+        CUDA_TRY(cudaGetLastError(), "dbuf_adam8_step_host: launch");
+        CUDA_TRY(cudaEventRecord(db->ev_step[i], st), "dbuf_adam8_step_host: record");
+        CUDA_TRY(cudaStreamWaitEvent(db->s_out, db->ev_step[i], 0), "dbuf_adam8_step_host: wait");
+        CUDA_TRY(cudaMemcpyAsync(ph + off, reinterpret_cast<const char*>(db->param) + off, len,
+                                 cudaMemcpyDeviceToHost, db->s_out),
+                 "dbuf_adam8_step_host: copy out");
+    }
+    CUDA_TRY(cudaEventRecord(db->ev_done, db->s_out), "dbuf_adam8_step_host: record");
+    CUDA_TRY(cudaStreamWaitEvent(st, db->ev_done, 0), "dbuf_adam8_step_host: wait");
     return DBUF_OK;
 }
 
