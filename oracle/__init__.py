@@ -2,8 +2,10 @@
 
 Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package.  It shares no code with the product
-library: the arithmetic lives in ``oracle.cpp`` (plain C++, fp32 in one fixed
-operation order) and this module only marshals numpy arrays.
+library.  The planner and the 8-bit Adam step live in ``oracle.cpp`` (plain
+C++, fp32 in one fixed operation order); this module marshals numpy arrays
+for them and holds, in plain numpy, the row-wise (FSDP2-style) baseline
+layout and the Muon pieces (fp32 momentum, float64 Newton-Schulz).
 
 Every function cites the part of the veScale-FSDP description it follows; the
 parity status of each is stated in ``oracle.cpp``'s header.

@@ -16,7 +16,9 @@
 //     one, and the bucket is cut into m equal per-device slices.
 //   * DBuffer (Sec. 5): the bucket is one flat buffer, tensors are views.
 //   * 8-bit Adam case study (Sec. 6.3): block-wise quantised optimizer states,
-//     each device quantising its own blocks without communication.
+//     each device quantising its own blocks without communication, with
+//     blocks of k whole rows or 2-D tiles (e.g. 32x32 elements) per
+//     parameter; a tile is gathered and stepped as one block.
 // The pages give no formulas for the quantiser or the update; the readings
 // taken here (linear absmax codes, int8 m, uint8 sqrt(v), decoupled weight
 // decay, round-half-even) are listed in the project's design notes.
@@ -28,8 +30,9 @@
 //
 // Parity status: layout and update are pinned by the CPU tests (literal
 // definition scans, exhaustive search on tiny instances, the closed-form first
-// step, code invariants, an fp64 shadow).  Parity with the pages' own system is
-// unpinned: the pages print no worked example.
+// step, code invariants, an fp64 shadow); the 2-D tile step by a worked first
+// step and by equality with the contiguous step on cut-out tiles.  Parity with
+// the pages' own system is unpinned: the pages print no worked example.
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
