@@ -270,8 +270,22 @@ def run_reference(args):
 
 # ------------------------------------------------------------ GPU arm
 
+def _ensure_library():
+    """Compile libdbuf.so with nvcc if this checkout has not built it yet (the
+    package itself refuses to load without it)."""
+    if os.path.exists(os.path.join(ROOT, "ragged_bucket_layout_b200", "libdbuf.so")):
+        return
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("_dbuf_build", os.path.join(ROOT, "ragged_bucket_layout_b200",
+                                                                              "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+
+
 def run_ours(args):
     import torch
+    _ensure_library()
     import ragged_bucket_layout_b200 as rb
 
     rank = int(os.environ.get("RANK", "0"))
