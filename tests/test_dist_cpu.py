@@ -74,3 +74,20 @@ def test_reference_arm_prints_the_contract_line():
     assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "GB/s"
     assert d["e2e"]["value"] == d["value"] and d["e2e"]["h2d_bytes_per_step"] == 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+
+
+def test_algorithmic_bytes_of_the_tiny_and_llama_buckets():
+    """16 B per parameter, 16 B per block, 2 B per padding element: the tiny
+    bucket (131,840 parameters, 34 blocks, 15,616 padding) moves 2,141,216 B
+    per step, the Llama bucket 3,490,693,152 B; copy-in moves 4 B per
+    parameter."""
+    import ragged_bucket_layout_b200 as rb
+    import synth
+    expect = {"tiny_m4": (131840, 34, 15616, 2141216), "llama_layer_m8": (218112000, 53250, 24576, 3490693152)}
+    for name, (P, B, pad, total) in expect.items():
+        w = synth.workload(name)
+        r, c, k = w.arrays()
+        info = rb.dbuf_plan_info(rb.dbuf_plan(r, c, k, w.m, 16))
+        st = bench.workload_stats(w, info)
+        assert (st["params"], st["blocks"], st["padding"], st["step_bytes"]) == (P, B, pad, total)
+        assert st["copy_in_bytes"] == 4 * P
