@@ -61,11 +61,16 @@ struct PosTiles {
     }
 };
 
-void add_zero_tiles(std::vector<Tile>& out, PosTiles* pos, int64_t a, int64_t b) {
-    for (int64_t e = a; e < b; e += kZeroChunk) {
-        const Tile t{e, 0, std::min(kZeroChunk, b - e), 0, TILE_ZERO, 0, 0u};
+// Padding [a, b) in entries of at most kZeroChunk elements, none crossing a
+// slice boundary (multiples of s; s = 0 means one slice).
+void add_zero_tiles(std::vector<Tile>& out, PosTiles* pos, int64_t a, int64_t b, int64_t s) {
+    for (int64_t e = a; e < b;) {
+        int64_t end = std::min(b, e + kZeroChunk);
+        if (s > 0) end = std::min(end, (e / s + 1) * s);
+        const Tile t{e, 0, end - e, 0, TILE_ZERO, 0, 0u};
         out.push_back(t);
         if (pos) pos->add(t, t.e0, t.e0 + t.n);
+        e = end;
     }
 }
 
@@ -78,7 +83,7 @@ void build_tiles(const dbuf_plan_s& p, std::vector<Tile>& tiles, PosTiles* pos =
     for (int32_t id : p.by_offset) {
         const int64_t o = p.offset[id], n = p.rows[id] * p.cols[id], b = p.k[id] * p.cols[id];
         const int64_t nb = cdiv(p.rows[id], p.k[id]);
-        if (o > prev_end) add_zero_tiles(zero, pos, prev_end, o);
+        if (o > prev_end) add_zero_tiles(zero, pos, prev_end, o, p.slice);
         if (!p.tile_cols.empty() && p.tile_cols[id] > 0) {
             // 2-D blocks: each k-row block in strips of at most kTile columns.
             const int64_t C = p.cols[id], W = p.tile_cols[id], G = cdiv(C, W);
@@ -99,7 +104,10 @@ void build_tiles(const dbuf_plan_s& p, std::vector<Tile>& tiles, PosTiles* pos =
             const int64_t e0 = o + j * b;
             if (b <= kTile) {
                 const int64_t cap = kTile - (e0 & (kAlign - 1));
-                const int64_t q = std::min<int64_t>({kMaxBlk, cap / b, nb - j});
+                // Every entry stays inside one rank's slice: blocks end on the
+                // slice boundary, so the blocks before it are whole.
+                const int64_t to_edge = p.slice > 0 ? ((e0 / p.slice + 1) * p.slice - e0) / b : nb - j;
+                const int64_t q = std::min<int64_t>({kMaxBlk, cap / b, nb - j, std::max<int64_t>(1, to_edge)});
                 if (q >= 1) {
                     const uint32_t magic = b >= 2 ? (uint32_t)(((uint64_t(1) << 32) + (uint64_t)b - 1) / (uint64_t)b) : 0u;
                     whole.push_back(Tile{e0, blk + j, std::min(q * b, n - j * b), (int32_t)b, TILE_WHOLE,
@@ -116,7 +124,7 @@ void build_tiles(const dbuf_plan_s& p, std::vector<Tile>& tiles, PosTiles* pos =
         blk += nb;
         prev_end = o + n;
     }
-    if (prev_end < p.bucket) add_zero_tiles(zero, pos, prev_end, p.bucket);
+    if (prev_end < p.bucket) add_zero_tiles(zero, pos, prev_end, p.bucket, p.slice);
     // Longest work first so the tail of the grid is short tiles.
     std::stable_sort(large.begin(), large.end(),
                      [](const Tile& x, const Tile& y) { return entry_work(x) > entry_work(y); });

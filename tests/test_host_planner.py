@@ -272,3 +272,21 @@ def test_plan_block_cols_rules(bc, cols, ok):
         with pytest.raises(rb.DbufError) as e:
             rb.dbuf_plan([64], [cols], [32], 2, 16, block_cols=[bc])
         assert e.value.status == rb.DBUF_EINVAL
+
+
+@pytest.mark.parametrize("name", ["tiny_m4", "llama_layer_m8", "moe_layer_m64", "ragged_stress_m8",
+                                  "ragged_stress_m128", "ragged_stress_m1024", "ragged_mix_m4", "ragged_mix_m8",
+                                  "tiles_mix_m4", "tiles_mix_m8", "llama_layer_32x32_m8"])
+def test_every_work_entry_lies_in_one_slice(name):
+    """RaggedShard's point: blocks never straddle a rank's slice, so each
+    rank can step its own slice with no exchange.  The work table keeps
+    that: every entry (padding entries too) lies inside one slice, so the
+    entries of slice r are exactly rank r's work."""
+    w = synth.workload(name)
+    r, c, k = w.arrays()
+    p = rb.dbuf_plan(r, c, k, w.m, 16, block_cols=w.block_cols())
+    s = rb.dbuf_plan_info(p)["slice"]
+    for t in rb.dbuf_work_table(p):
+        lo = t["first_elem"]
+        hi = lo + ((t["n_blocks"] - 1) * t["block_elems"] + t["n_elems"] if t["kind"] == 3 else t["n_elems"])
+        assert lo // s == (hi - 1) // s, t
