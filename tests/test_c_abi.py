@@ -1,0 +1,37 @@
+"""The C-ABI from plain C99: tests/c_abi_check.c includes only include/dbuf.h,
+links libdbuf.so, and calls the host-only entry points (planner, work
+table, required bytes, row-wise layout, error path).  Its numbers must
+equal what the Python binding reports (CPU only)."""
+import os
+import re
+import subprocess
+
+import ragged_bucket_layout_b200 as rb
+import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_c99_caller(tmp_path):
+    exe = tmp_path / "c_abi_check"
+    libdir = os.path.dirname(rb.LIB_PATH)
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                           "-o", str(exe), os.path.join(ROOT, "tests", "c_abi_check.c"), "-L", libdir, "-ldbuf",
+                           f"-Wl,-rpath,{libdir}"])
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, out.stdout + out.stderr
+    w = synth.workload("tiny_m4")
+    r, c, k = w.arrays()
+    p = rb.dbuf_plan(r, c, k, w.m, 16)
+    info = rb.dbuf_plan_info(p)
+    m = re.search(r"slice=(\d+) bucket=(\d+) padding=(\d+) n_blocks=(\d+) offsets=(\d+),(\d+),(\d+)", out.stdout)
+    assert m, out.stdout
+    assert [int(x) for x in m.groups()] == [info["slice"], info["bucket"], info["padding"], info["n_blocks"],
+                                            *info["offsets"]]
+    m = re.search(r"entries=(\d+) covered=(\d+) required_bytes=(\d+)", out.stdout)
+    assert int(m.group(1)) == len(rb.dbuf_work_table(p))
+    assert int(m.group(2)) == info["bucket"]
+    assert int(m.group(3)) == rb.dbuf_required_bytes(p)
+    assert re.search(r"bad=%d msg_nonempty=1" % rb.DBUF_EINVAL, out.stdout), out.stdout
+    chunk, q, _ = rb.dbuf_rowwise_layout(r, c, 4)
+    assert f"rowwise chunk={chunk} q={q[0]},{q[1]},{q[2]}" in out.stdout
