@@ -35,3 +35,24 @@ def test_c99_caller(tmp_path):
     assert re.search(r"bad=%d msg_nonempty=1" % rb.DBUF_EINVAL, out.stdout), out.stdout
     chunk, q, _ = rb.dbuf_rowwise_layout(r, c, 4)
     assert f"rowwise chunk={chunk} q={q[0]},{q[1]},{q[2]}" in out.stdout
+
+
+import pytest  # noqa: E402
+
+
+@pytest.mark.gpu
+def test_c99_caller_on_the_device(tmp_path):
+    """Plain C99 drives the whole device path: library-allocated bucket,
+    resident step, host-buffer step, status word."""
+    exe = tmp_path / "c_abi_gpu"
+    libdir = os.path.dirname(rb.LIB_PATH)
+    cuda = "/usr/local/cuda"
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                           "-I", os.path.join(cuda, "include"), "-o", str(exe),
+                           os.path.join(ROOT, "tests", "c_abi_gpu.c"), "-L", libdir, "-ldbuf",
+                           "-L", os.path.join(cuda, "lib64"), "-lcudart", "-lm", f"-Wl,-rpath,{libdir}"])
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0, out.stdout + out.stderr
+    m = re.search(r"first_step_worst_abs_err=(\S+) second_step_param=(\S+) status=(\d+)", out.stdout)
+    assert m and float(m.group(1)) < 1e-6 and int(m.group(3)) == 0, out.stdout
+    assert 0.0075 < float(m.group(2)) < 0.0085     # two steps of about lr each from 0.01
