@@ -97,6 +97,18 @@ dbuf_status dbuf_plan_info(const dbuf_plan_t* plan, int64_t* slice_elems, int64_
 
 void dbuf_plan_free(dbuf_plan_t* plan); /* NULL is a no-op */
 
+/* RaggedShard placement of a plan (paper Sec. 3; page section
+ * "1. RaggedShard": devices hold different numbers of whole blocks): the
+ * rows of each tensor that each rank's slice holds.  out[i*m + r] (host
+ * array of n*m entries) gets rows [row_begin, row_end) of tensor i in slice
+ * r, an empty range when it holds none.  The ranges of a tensor increase with
+ * r and cover all its rows, and every boundary between two ranks is a k-row
+ * block edge, so each rank quantises its own blocks.  Host only. */
+typedef struct {
+    int64_t row_begin, row_end;
+} dbuf_shard_rows;
+dbuf_status dbuf_plan_shards(const dbuf_plan_t* plan, dbuf_shard_rows* out);
+
 /* Bytes of device memory dbuf_create needs for this plan (one allocation:
  * fp32 master, bf16 param, bf16 grad, int8 m codes, uint8 sqrt(v) codes,
  * per-block scales, work tables, status word), 256-byte aligned parts.

@@ -187,6 +187,24 @@ def tiles(rows, cols, k, block_cols, offsets):
     return mk(base), mk(trows), mk(width), mk(stride)
 
 
+def shards(rows, cols, offsets, s, m):
+    """RaggedShard placement (paper Sec. 3; devices hold different numbers of
+    whole blocks): for each tensor and rank, the rows [begin, end) of the
+    tensor that lie in slice r = [r s, (r+1) s) of the bucket."""
+    out = []
+    for R, C, o in zip(_i64(rows), _i64(cols), _i64(offsets)):
+        per = []
+        for r in range(m):
+            lo, hi = max(int(o), r * s), min(int(o) + int(R * C), (r + 1) * s)
+            if hi <= lo:
+                first = min(int(R), max(0, -(-(r * s - int(o)) // int(C))))
+                per.append((first, first))
+            else:
+                per.append(((lo - int(o)) // int(C), (hi - int(o)) // int(C)))
+        out.append(per)
+    return out
+
+
 def padding_mask(rows, cols, offsets, bucket):
     """Boolean mask of bucket elements that belong to no tensor."""
     mask = np.ones(bucket, dtype=bool)

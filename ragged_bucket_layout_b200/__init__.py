@@ -60,6 +60,7 @@ _SIGS = {
     "dbuf_plan": (ctypes.c_int, [ctypes.POINTER(dbuf_tensor_desc), _i32, _i32, _i64, _i64, _PP]),
     "dbuf_plan_info": (ctypes.c_int, [_P, _pi64, _pi64, _pi64, _pi64, _pi64]),
     "dbuf_plan_free": (None, [_P]),
+    "dbuf_plan_shards": (ctypes.c_int, [_P, _P]),
     "dbuf_required_bytes": (_sz, [_P]),
     "dbuf_create": (ctypes.c_int, [_P, _P, _sz, _P, _PP]),
     "dbuf_pack_grads": (ctypes.c_int, [_P, _PP, _f32, _P]),
@@ -150,6 +151,13 @@ def dbuf_plan_info(plan):
                                ctypes.byref(nb), offs))
     return dict(slice=s.value, bucket=b.value, padding=p.value, n_blocks=nb.value,
                 offsets=[offs[i] for i in range(plan.n)])
+
+
+def dbuf_plan_shards(plan, m):
+    """RaggedShard placement: [[(row_begin, row_end) for each rank] for each tensor]."""
+    arr = (ctypes.c_int64 * max(2 * plan.n * m, 1))()
+    _check(_lib.dbuf_plan_shards(plan.handle, arr))
+    return [[(arr[2 * (i * m + r)], arr[2 * (i * m + r) + 1]) for r in range(m)] for i in range(plan.n)]
 
 
 def dbuf_plan_free(plan):

@@ -211,4 +211,21 @@ extern "C" dbuf_status dbuf_plan_info(const dbuf_plan_t* plan, int64_t* slice_el
     return DBUF_OK;
 }
 
+extern "C" dbuf_status dbuf_plan_shards(const dbuf_plan_t* plan, dbuf_shard_rows* out) {
+    if (!plan) return dbuf_detail::fail(DBUF_EINVAL, "dbuf_plan_shards: plan is NULL");
+    if (plan->n > 0 && !out) return dbuf_detail::fail(DBUF_EINVAL, "dbuf_plan_shards: out is NULL");
+    const int64_t s = plan->slice;
+    for (int32_t i = 0; i < plan->n; ++i) {
+        const int64_t o = plan->offset[i], c = plan->cols[i], n = plan->rows[i] * c;
+        for (int32_t r = 0; r < plan->m; ++r) {
+            // The part of the tensor inside slice r, in elements from its start;
+            // interior slice boundaries are block edges, so whole rows.
+            const int64_t a = std::min(n, std::max<int64_t>(0, (int64_t)r * s - o));
+            const int64_t b = std::min(n, std::max<int64_t>(0, (int64_t)(r + 1) * s - o));
+            out[(int64_t)i * plan->m + r] = dbuf_shard_rows{a / c, std::max(a, b) / c};
+        }
+    }
+    return DBUF_OK;
+}
+
 extern "C" void dbuf_plan_free(dbuf_plan_t* plan) { delete plan; }

@@ -290,3 +290,37 @@ def test_every_work_entry_lies_in_one_slice(name):
         lo = t["first_elem"]
         hi = lo + ((t["n_blocks"] - 1) * t["block_elems"] + t["n_elems"] if t["kind"] == 3 else t["n_elems"])
         assert lo // s == (hi - 1) // s, t
+
+
+@pytest.mark.parametrize("name", ["tiny_m4", "llama_layer_m8", "moe_layer_m64", "ragged_stress_m128",
+                                  "ragged_stress_m1024", "ragged_mix_m4", "ragged_mix_m8", "tiles_mix_m8"])
+def test_plan_shards_match_oracle_and_keep_blocks_whole(name):
+    """dbuf_plan_shards equals the oracle's placement; every tensor's rows
+    are covered once, in rank order, and each boundary between two ranks
+    is a k-row block edge (RaggedShard: a block is never split)."""
+    w = synth.workload(name)
+    r, c, k = w.arrays()
+    p = rb.dbuf_plan(r, c, k, w.m, 16, block_cols=w.block_cols())
+    info = rb.dbuf_plan_info(p)
+    got = rb.dbuf_plan_shards(p, w.m)
+    assert got == oracle.shards(r, c, info["offsets"], info["slice"], w.m)
+    for i, per in enumerate(got):
+        assert per[0][0] == 0 and per[-1][1] == r[i]
+        for (b0, e0), (b1, e1) in zip(per, per[1:]):
+            assert b0 <= e0 == b1 <= e1
+        for b, e in per:
+            if e > b:
+                assert b % k[i] == 0 and (e % k[i] == 0 or e == r[i])
+
+
+def test_oracle_shards_against_per_element_slices():
+    """Brute force on the ragged mix: assign every bucket element its slice
+    and count each tensor's elements per slice."""
+    w = synth.workload("ragged_mix_m4")
+    r, c, k = w.arrays()
+    st, off, s = oracle.plan(r, c, k, w.m, 16)
+    sh = oracle.shards(r, c, off, s, w.m)
+    for i in range(len(r)):
+        e = int(off[i]) + np.arange(int(r[i] * c[i]))
+        counts = np.bincount(e // s, minlength=w.m)
+        assert [(hi - lo) * int(c[i]) for lo, hi in sh[i]] == counts.tolist()
