@@ -388,9 +388,32 @@ def run_ours(args):
         e1.synchronize()
         barrier()
         ems = max_over_ranks(e0.elapsed_time(e1), dist, "cuda") / args.e2e_steps
+        # The PCIe bound of this path: the same bytes copied in and out at
+        # once, pinned, with nothing else running.
+        d_in = torch.empty(S, dtype=torch.int16, device="cuda")
+        d_out = torch.empty(S, dtype=torch.int16, device="cuda")
+        h_back = torch.empty(S, dtype=torch.int16).pin_memory()
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+
+        def both_ways():
+            with torch.cuda.stream(s_in):
+                d_in.copy_(g_host, non_blocking=True)
+            with torch.cuda.stream(s_out):
+                h_back.copy_(d_out, non_blocking=True)
+            s_in.synchronize()
+            s_out.synchronize()
+        both_ways()
+        t0 = time.perf_counter()
+        for _ in range(3):
+            both_ways()
+        pcie_ms = (time.perf_counter() - t0) / 3 * 1e3
+        ceiling = stats["step_bytes"] / (pcie_ms * 1e-3) / 1e9
         e2e = {"value": world * stats["step_bytes"] / (ems * 1e-3) / 1e9, "unit": UNIT,
                "h2d_bytes_per_step": 2 * S, "d2h_bytes_per_step": 2 * S, "ms_per_step": ems,
-               "path": "dbuf_adam8_step_host (pinned host grads in, bf16 params out)"}
+               "path": "dbuf_adam8_step_host (pinned host grads in, bf16 params out)",
+               "pcie_bound": {"copy_in_and_out_ms": pcie_ms, "ceiling_gbs": ceiling,
+                              "frac": (stats["step_bytes"] / (ems * 1e-3) / 1e9) / ceiling}}
+        del d_in, d_out, h_back
 
     # ---- copy-in baseline on the same workload (rank-local, informative)
     copy_in = None
