@@ -109,6 +109,23 @@ typedef struct {
 } dbuf_shard_rows;
 dbuf_status dbuf_plan_shards(const dbuf_plan_t* plan, dbuf_shard_rows* out);
 
+/* The bucket one rank holds, as a plan of its own (page section "1.
+ * RaggedShard" and paper Sec. 3: each device quantises the whole blocks of
+ * its slice, with no exchange): slice `rank` = [rank*s, (rank+1)*s) of the
+ * bucket, with m = 1 and slice = bucket = s.  Its tensors are the non-empty
+ * row ranges dbuf_plan_shards gives for that rank, in the parent's caller
+ * order (tensors with no rows there are left out). Each range keeps cols,
+ * k and block_cols and sits at its parent offset minus rank*s; a range
+ * shorter than k rows is the tensor's last block.  Its blocks are the parent's
+ * blocks inside the slice in the same order, so a dbuf created from it, given
+ * slice `rank` of the gradient bucket and stepped with the same
+ * hyperparameters and grad_scale, holds slice `rank` of the parent's bucket
+ * bit for bit. It stores the fp32 master weights, codes and scales of that
+ * one slice only.  *first_block (may be NULL) receives the parent's index of
+ * its block 0.  rank in [0, m); *out (freed with dbuf_plan_free) is NULL on
+ * failure.  Host only. */
+dbuf_status dbuf_plan_rank(const dbuf_plan_t* plan, int32_t rank, dbuf_plan_t** out, int64_t* first_block);
+
 /* Bytes of device memory dbuf_create needs for this plan (one allocation:
  * fp32 master, bf16 param, bf16 grad, int8 m codes, uint8 sqrt(v) codes,
  * per-block scales, work tables, status word), 256-byte aligned parts.

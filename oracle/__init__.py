@@ -205,6 +205,49 @@ def shards(rows, cols, offsets, s, m):
     return out
 
 
+def rank_bucket(rows, cols, k, offsets, s, m, r, block_cols=None):
+    """The part of a bucket that rank r holds (paper Sec. 3; each device
+    quantises the whole blocks of its own slice [r s, (r+1) s)), described
+    as a bucket of its own with one slice of s elements.
+
+    Each tensor's elements [o, o + rows*cols) are intersected with the slice;
+    a non-empty intersection is whole rows (interior slice boundaries are
+    block edges) and becomes a tensor of those rows, same cols, k and
+    block_cols, at its offset minus r s.  Returns a dict with the parts
+    (parent id, row_begin, row_end) in parent order, their rows, cols, k,
+    block_cols and offsets, and first_block, the number of the parent's
+    quantisation blocks (numbered in bucket order) that come before the
+    slice.
+    """
+    rows, cols, k, off = _i64(rows), _i64(cols), _i64(k), _i64(offsets)
+    bc = _i64(block_cols) if block_cols is not None else np.zeros_like(rows)
+    lo, hi = int(r) * int(s), (int(r) + 1) * int(s)
+    out = dict(parts=[], rows=[], cols=[], k=[], block_cols=[], offsets=[])
+    first_block = 0
+    for i in range(rows.size):
+        R, C, K, o = int(rows[i]), int(cols[i]), int(k[i]), int(off[i])
+        tiles_per_row_block = 1 if bc[i] <= 0 or bc[i] >= C else -(-C // int(bc[i]))
+        a, b = max(o, lo), min(o + R * C, hi)
+        # Row blocks of the tensor that start before the slice.
+        first_row_in = R if o + R * C <= lo else max(0, lo - o) // C
+        first_block += tiles_per_row_block * (-(-first_row_in // K))
+        if b <= a:
+            continue
+        assert (a - o) % C == 0 and (b - o) % C == 0, "a slice boundary cuts a row"
+        assert ((a - o) // C) % K == 0, "a slice boundary cuts a block"
+        out["parts"].append((i, (a - o) // C, (b - o) // C))
+        out["rows"].append((b - a) // C)
+        out["cols"].append(C)
+        out["k"].append(K)
+        out["block_cols"].append(int(bc[i]))
+        out["offsets"].append(a - lo)
+    for key in ("rows", "cols", "k", "block_cols", "offsets"):
+        out[key] = np.asarray(out[key], dtype=np.int64)
+    out["first_block"] = first_block
+    out["s"] = int(s)
+    return out
+
+
 def padding_mask(rows, cols, offsets, bucket):
     """Boolean mask of bucket elements that belong to no tensor."""
     mask = np.ones(bucket, dtype=bool)

@@ -31,7 +31,10 @@
 // Parity status: layout and update are pinned by the CPU tests (literal
 // definition scans, exhaustive search on tiny instances, the closed-form first
 // step, code invariants, an fp64 shadow); the 2-D tile step by a worked first
-// step and by equality with the contiguous step on cut-out tiles.  Parity with
+// step and by equality with the contiguous step on cut-out tiles.  The rank
+// buckets (rank_bucket in __init__.py: one slice as a bucket of its own) are
+// pinned by stepping every rank's bucket alone and finding the whole bucket's
+// result bit for bit, and by their parts tiling every tensor.  Parity with
 // the pages' own system is unpinned: the pages print no worked example.
 #include <algorithm>
 #include <cmath>

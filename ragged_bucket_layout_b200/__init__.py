@@ -61,6 +61,7 @@ _SIGS = {
     "dbuf_plan_info": (ctypes.c_int, [_P, _pi64, _pi64, _pi64, _pi64, _pi64]),
     "dbuf_plan_free": (None, [_P]),
     "dbuf_plan_shards": (ctypes.c_int, [_P, _P]),
+    "dbuf_plan_rank": (ctypes.c_int, [_P, _i32, _PP, _pi64]),
     "dbuf_required_bytes": (_sz, [_P]),
     "dbuf_create": (ctypes.c_int, [_P, _P, _sz, _P, _PP]),
     "dbuf_pack_grads": (ctypes.c_int, [_P, _PP, _f32, _P]),
@@ -121,9 +122,10 @@ def _stream(s):
 class Plan:
     """Owner of a dbuf_plan_t (freed with dbuf_plan_free)."""
 
-    def __init__(self, handle, n):
+    def __init__(self, handle, n, m=None):
         self.handle = handle
         self.n = n
+        self.m = m
         self._free = _lib.dbuf_plan_free   # held here: module globals may be gone at interpreter exit
 
     def __del__(self):
@@ -141,7 +143,9 @@ def dbuf_plan(rows, cols, k, m, align_elems=16, max_bucket_elems=0, block_cols=N
                                              for r, c, q, b in zip(rows, cols, k, bc)])
     out = ctypes.c_void_p()
     _check(_lib.dbuf_plan(descs, n, int(m), int(align_elems), int(max_bucket_elems), ctypes.byref(out)))
-    return Plan(out.value, n)
+    plan = Plan(out.value, n, int(m))
+    plan.shapes = [(int(r), int(c)) for r, c in zip(rows, cols)]
+    return plan
 
 
 def dbuf_plan_info(plan):
@@ -158,6 +162,23 @@ def dbuf_plan_shards(plan, m):
     arr = (ctypes.c_int64 * max(2 * plan.n * m, 1))()
     _check(_lib.dbuf_plan_shards(plan.handle, arr))
     return [[(arr[2 * (i * m + r)], arr[2 * (i * m + r) + 1]) for r in range(m)] for i in range(plan.n)]
+
+
+def dbuf_plan_rank(plan, rank):
+    """The bucket rank `rank` holds, as a plan of its own (m = 1, bucket =
+    one slice).  The result also carries `rank`, `first_block` (the parent's
+    index of its block 0) and `parts`: for each of its tensors, in order,
+    (parent tensor id, row_begin, row_end)."""
+    if plan.m is None:
+        raise ValueError("dbuf_plan_rank needs a plan made by dbuf_plan (m unknown)")
+    out, fb = ctypes.c_void_p(), ctypes.c_int64()
+    _check(_lib.dbuf_plan_rank(plan.handle, int(rank), ctypes.byref(out), ctypes.byref(fb)))
+    parts = [(i, a, b) for i, per in enumerate(dbuf_plan_shards(plan, plan.m)) for a, b in [per[rank]] if b > a]
+    sub = Plan(out.value, len(parts), 1)
+    sub.rank, sub.first_block, sub.parts = int(rank), fb.value, parts
+    if getattr(plan, "shapes", None) is not None:
+        sub.shapes = [(b - a, plan.shapes[i][1]) for i, a, b in parts]
+    return sub
 
 
 def dbuf_plan_free(plan):

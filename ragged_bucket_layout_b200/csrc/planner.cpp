@@ -228,4 +228,55 @@ extern "C" dbuf_status dbuf_plan_shards(const dbuf_plan_t* plan, dbuf_shard_rows
     return DBUF_OK;
 }
 
+extern "C" dbuf_status dbuf_plan_rank(const dbuf_plan_t* plan, int32_t rank, dbuf_plan_t** out,
+                                      int64_t* first_block) {
+    using dbuf_detail::fail;
+    if (!out) return fail(DBUF_EINVAL, "dbuf_plan_rank: out is NULL");
+    *out = nullptr;
+    if (!plan) return fail(DBUF_EINVAL, "dbuf_plan_rank: plan is NULL");
+    if (rank < 0 || rank >= plan->m) return fail(DBUF_EINVAL, "dbuf_plan_rank: rank must be in [0, m)");
+    dbuf_plan_s* p = new (std::nothrow) dbuf_plan_s;
+    if (!p) return fail(DBUF_ENOMEM, "dbuf_plan_rank: out of host memory");
+    const int64_t s = plan->slice, lo = (int64_t)rank * s, hi = lo + s;
+    int64_t used = 0, nb = 0, before = 0;
+    for (int32_t i = 0; i < plan->n; ++i) {
+        const int64_t o = plan->offset[i], c = plan->cols[i], K = plan->k[i], n = plan->rows[i] * c;
+        const int64_t tc = plan->tile_cols.empty() ? 0 : plan->tile_cols[i];
+        const int64_t G = tc ? cdiv(c, tc) : 1;  // blocks per k-row block
+        // Elements [a, b) of the tensor lie in the slice.  Interior slice
+        // boundaries are k-row block edges, so both are whole rows and a is a
+        // multiple of k rows.
+        const int64_t a = std::min(n, std::max<int64_t>(0, lo - o));
+        const int64_t b = std::max(a, std::min(n, std::max<int64_t>(0, hi - o)));
+        if (a % c != 0 || b % c != 0 || (a < n && (a / c) % K != 0)) {
+            delete p;
+            return fail(DBUF_EINVAL, "dbuf_plan_rank: tensor " + std::to_string(i) +
+                                         " is cut off a block edge (not a plan from dbuf_plan)");
+        }
+        before += G * cdiv(a / c, K);
+        if (b == a) continue;
+        p->rows.push_back((b - a) / c);
+        p->cols.push_back(c);
+        p->k.push_back(K);
+        p->tile_cols.push_back(tc);
+        p->offset.push_back(o + a - lo);
+        used += b - a;
+        nb += G * cdiv((b - a) / c, K);
+    }
+    p->n = (int32_t)p->rows.size();
+    p->m = 1;
+    p->align = plan->align;
+    p->slice = s;
+    p->bucket = s;
+    p->padding = s - used;
+    p->n_blocks = nb;
+    p->by_offset.resize(p->n);
+    std::iota(p->by_offset.begin(), p->by_offset.end(), 0);
+    std::stable_sort(p->by_offset.begin(), p->by_offset.end(),
+                     [&](int32_t x, int32_t y) { return p->offset[x] < p->offset[y]; });
+    if (first_block) *first_block = before;
+    *out = p;
+    return DBUF_OK;
+}
+
 extern "C" void dbuf_plan_free(dbuf_plan_t* plan) { delete plan; }

@@ -1,0 +1,92 @@
+"""One rank's side of a data-parallel bucket step over the RaggedShard layout.
+
+veScale-FSDP (paper Sec. 3 and Sec. 5; page sections "1. RaggedShard" and
+"3. DBuffer"): the gradient bucket is reduce-scattered so that rank r gets
+slice r = [r s, (r+1) s); rank r runs the 8-bit Adam step over the whole
+blocks of that slice alone (no block straddles a slice, so the step itself
+exchanges nothing); the bf16 parameters are all-gathered back into the full
+bucket, where every tensor is a view at its planned offset.
+
+Per rank this holds:
+  * the full bf16 gradient and parameter buckets, m*s elements each: the
+    buffers the two collectives work on, tensors as zero-copy views;
+  * a bucket of one slice (dbuf_plan_rank) with this rank's fp32 master
+    weights, 8-bit codes and scales: 1/m of the optimizer state.
+The collectives are torch.distributed's (NCCL between GPUs), issued on the
+slice bucket's stream; the step is the library's fused kernel.  With
+async_op the all-gather is left in flight, so the next bucket's
+reduce-scatter and step can be queued behind it.
+"""
+import contextlib
+
+from . import (DBUF_GRAD_BF16, DBUF_PARAM_BF16, DBuffer, dbuf_plan_info, dbuf_plan_rank)
+
+
+class ShardedBucket:
+    """Rank `rank` of `world` for the bucket of `plan` (planned with
+    m = world).  `local` replaces the slice bucket (a DBuffer of
+    dbuf_plan_rank(plan, rank) on `device` by default) with any object that
+    has array(which), views(which) and step(hp, grad_scale), e.g. a host-side
+    model of it."""
+
+    def __init__(self, plan, rank=None, world=None, group=None, device="cuda", local=None):
+        import torch
+        import torch.distributed as dist
+
+        self.group = group
+        self.rank = dist.get_rank(group) if rank is None else int(rank)
+        self.world = dist.get_world_size(group) if world is None else int(world)
+        if plan.m != self.world:
+            raise ValueError(f"the plan has {plan.m} slices for {self.world} ranks")
+        if getattr(plan, "shapes", None) is None:
+            raise ValueError("ShardedBucket needs a plan made by dbuf_plan")
+        self.plan = plan
+        self.rank_plan = dbuf_plan_rank(plan, self.rank)
+        info = dbuf_plan_info(plan)
+        self.slice, self.offsets = info["slice"], info["offsets"]
+        self.local = DBuffer(self.rank_plan, device=device) if local is None else local
+        dev = self.local.array(DBUF_GRAD_BF16).device
+        with self._on_stream():
+            self.grad = torch.zeros(info["bucket"], dtype=torch.bfloat16, device=dev)
+            self.param = torch.zeros(info["bucket"], dtype=torch.bfloat16, device=dev)
+
+    def _on_stream(self):
+        import torch
+        s = getattr(self.local, "stream", None)
+        return torch.cuda.stream(s) if s is not None else contextlib.nullcontext()
+
+    def _full_views(self, flat):
+        return [flat[o:o + r * c].view(r, c) for o, (r, c) in zip(self.offsets, self.plan.shapes)]
+
+    def grad_views(self):
+        """Each tensor's gradient in the full bucket (where backward writes)."""
+        return self._full_views(self.grad)
+
+    def param_views(self):
+        """Each tensor's bf16 parameters in the full bucket (the forward's
+        weights; filled by the all-gather)."""
+        return self._full_views(self.param)
+
+    def local_views(self, which):
+        """This rank's rows of each tensor in the slice bucket:
+        [(tensor id, row_begin, row_end, view)] for the tensors it holds."""
+        return [(i, a, b, v) for (i, a, b), v in zip(self.rank_plan.parts, self.local.views(which))]
+
+    def all_gather_params(self, async_op=False):
+        """Gather every rank's bf16 slice into the full parameter bucket."""
+        import torch.distributed as dist
+        with self._on_stream():
+            return dist.all_gather_into_tensor(self.param, self.local.array(DBUF_PARAM_BF16), group=self.group,
+                                               async_op=async_op)
+
+    def step(self, hp, grad_scale=None, async_op=False):
+        """Reduce-scatter (sum) the gradient bucket into this rank's slice,
+        step the slice with grad_scale (default 1/world: the mean), then
+        all-gather the bf16 slices.  Returns the all-gather's work handle
+        when async_op is set."""
+        import torch.distributed as dist
+        gs = 1.0 / self.world if grad_scale is None else float(grad_scale)
+        with self._on_stream():
+            dist.reduce_scatter_tensor(self.local.array(DBUF_GRAD_BF16), self.grad, group=self.group)
+            self.local.step(hp, gs)
+        return self.all_gather_params(async_op=async_op)

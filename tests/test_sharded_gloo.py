@@ -1,0 +1,145 @@
+"""The per-rank bucket step (ShardedBucket) with real processes on CPU.
+
+Each rank: its own gradients into the full bucket -> reduce-scatter (gloo,
+sum) into its slice -> step of the slice alone -> all-gather of the bf16
+slices.  The slice bucket is stepped by the oracle here (there is no GPU),
+so this checks the collective plumbing and the per-rank layout around the
+step: every rank must end with the whole-bucket oracle step's bf16 bucket,
+and rank r with slice r of its master weights, codes and scales.
+
+Gradients are small multiples of 2^-8 (at most 64 in size), so their sum
+over up to four ranks is exact in bf16 whatever order the reduction takes.
+"""
+import datetime
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+CASES = {
+    # W[512,256] in 16-row blocks, bias and norm as one block each
+    "tiny": ([512, 512, 256], [256, 1, 1], [16, 512, 256], [0, 0, 0]),
+    # 2-D blocks cut by slice boundaries, a short last block, a 1-D tensor
+    "tiles": ([96, 40, 100, 5], [64, 32, 32, 16], [8, 4, 16, 5], [16, 16, 0, 0]),
+    # one tensor that leaves most slices empty
+    "empty": ([1000, 48], [1, 16], [1000, 48], [0, 0]),
+}
+STEPS = 3
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _hp(t):
+    return dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01, step=t)
+
+
+def _master(rows, cols):
+    rng = np.random.default_rng(7)
+    return [rng.normal(0.0, 0.02, size=(r, c)).astype(np.float32) for r, c in zip(rows, cols)]
+
+
+def _grad(rows, cols, rank, t):
+    """Rank `rank`'s gradients at step t (float32, exact in bf16)."""
+    rng = np.random.default_rng(1000 * t + rank)
+    return [(rng.integers(-64, 65, size=(r, c)) * 2.0 ** -8).astype(np.float32) for r, c in zip(rows, cols)]
+
+
+def _bf16_bits(x):
+    bits = np.ascontiguousarray(x, np.float32).view(np.uint32)
+    assert not np.any(bits & 0xFFFF), "value not exact in bf16"
+    return (bits >> 16).astype(np.uint16)
+
+
+class OracleSlice:
+    """The slice bucket of one rank, held and stepped by the oracle."""
+
+    def __init__(self, rk):
+        import oracle
+        self.rk = rk
+        self.b = oracle.Bucket(rk["rows"], rk["cols"], rk["k"], rk["offsets"], rk["s"], 1,
+                               block_cols=rk["block_cols"])
+        self.stream = None
+
+    def array(self, which):
+        a = {0: self.b.p, 1: self.b.pb, 2: self.b.g, 3: self.b.mq, 4: self.b.vq}[which]
+        t = torch.from_numpy(a)
+        return t.view(torch.int16).view(torch.bfloat16) if a.dtype == np.uint16 else t
+
+    def views(self, which):
+        flat = self.array(which)
+        return [flat[int(o):int(o) + int(r * c)].view(int(r), int(c))
+                for r, c, o in zip(self.rk["rows"], self.rk["cols"], self.rk["offsets"])]
+
+    def step(self, hp, grad_scale):
+        self.b.step(hp, hp["step"], grad_scale)
+
+
+def _worker(rank, world, port, case, outdir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        import oracle
+        import ragged_bucket_layout_b200 as rb
+        from ragged_bucket_layout_b200.sharded import ShardedBucket
+
+        rows, cols, k, bc = CASES[case]
+        plan = rb.dbuf_plan(rows, cols, k, world, 16, block_cols=bc)
+        info = rb.dbuf_plan_info(plan)
+        local = OracleSlice(oracle.rank_bucket(rows, cols, k, info["offsets"], info["slice"], world, rank, bc))
+        sb = ShardedBucket(plan, local=local)
+        assert (sb.rank, sb.world) == (rank, world)
+        full = _master(rows, cols)
+        for i, a, b, v in sb.local_views(rb.DBUF_MASTER_F32):
+            v.copy_(torch.from_numpy(full[i][a:b]))
+        for t in range(1, STEPS + 1):
+            for g, x in zip(sb.grad_views(), _grad(rows, cols, rank, t)):
+                g.copy_(torch.from_numpy(x))
+            work = sb.step(_hp(t), async_op=(t == STEPS))
+            if work is not None:
+                work.wait()
+        np.savez(os.path.join(outdir, f"rank{rank}.npz"), param=sb.param.view(torch.int16).numpy(),
+                 p=local.b.p, mq=local.b.mq, vq=local.b.vq, sm=local.b.scale_m, sv=local.b.scale_v,
+                 first_block=sb.rank_plan.first_block, n=sb.rank_plan.n)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("case,world", [("tiny", 2), ("tiny", 4), ("tiles", 2), ("tiles", 4), ("empty", 4)])
+def test_sharded_step_equals_the_whole_bucket(case, world, tmp_path):
+    import oracle
+
+    mp.start_processes(_worker, args=(world, _free_port(), case, str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    rows, cols, k, bc = CASES[case]
+    st, off, s = oracle.plan(rows, cols, k, world, 16)
+    assert st == 0
+    W = oracle.Bucket(rows, cols, k, off, s, world, block_cols=bc)
+    for i, x in enumerate(_master(rows, cols)):
+        W.p[W.tensor_slice(i)] = x.ravel()
+    for t in range(1, STEPS + 1):
+        per_rank = [_grad(rows, cols, r, t) for r in range(world)]
+        for i in range(len(rows)):
+            W.g[W.tensor_slice(i)] = _bf16_bits(sum(g[i] for g in per_rank).ravel())
+        W.step(_hp(t), t, 1.0 / world)
+    parts = 0
+    for r in range(world):
+        got = np.load(tmp_path / f"rank{r}.npz")
+        sl = slice(r * s, (r + 1) * s)
+        assert np.array_equal(got["param"].view(np.uint16), W.pb), f"rank {r}: gathered bf16 bucket"
+        assert np.array_equal(got["p"].view(np.uint32), W.p[sl].view(np.uint32)), f"rank {r}: master"
+        assert np.array_equal(got["mq"], W.mq[sl]) and np.array_equal(got["vq"], W.vq[sl]), f"rank {r}: codes"
+        fb, nb = int(got["first_block"]), got["sm"].size
+        assert np.array_equal(got["sm"], W.scale_m[fb:fb + nb]) and np.array_equal(got["sv"], W.scale_v[fb:fb + nb])
+        parts += int(got["n"])
+    assert parts >= len(rows)
+    if case == "empty":
+        assert any(int(np.load(tmp_path / f"rank{r}.npz")["n"]) == 0 for r in range(world))
