@@ -18,6 +18,8 @@ async_op the all-gather is left in flight, so the next bucket's
 reduce-scatter and step can be queued behind it.
 """
 import contextlib
+import ctypes
+import math
 
 from . import (DBUF_GRAD_BF16, DBUF_PARAM_BF16, DBuffer, dbuf_plan_info, dbuf_plan_rank)
 
@@ -79,14 +81,44 @@ class ShardedBucket:
             return dist.all_gather_into_tensor(self.param, self.local.array(DBUF_PARAM_BF16), group=self.group,
                                                async_op=async_op)
 
+    def _reduce_scatter(self):
+        import torch.distributed as dist
+        dist.reduce_scatter_tensor(self.local.array(DBUF_GRAD_BF16), self.grad, group=self.group)
+
+    def step_clipped(self, hp, max_norm, grad_scale=None, async_op=False):
+        """step() with global-norm clipping over the whole bucket, as the
+        single-bucket dbuf_adam8_step_clipped does it:
+        grad_scale * min(1, max_norm / (norm + 1e-6)), formed in double and
+        rounded to float once.  Each rank takes its slice's norm with the
+        library's grad-norm kernel, and an all-reduce sums the squares.
+        The coefficient is formed on the host, so this waits for the
+        reduce-scatter and the norm.  Returns (norm, all-gather handle or
+        None)."""
+        import torch
+        import torch.distributed as dist
+        gs = ctypes.c_float(1.0 / self.world if grad_scale is None else float(grad_scale)).value
+        mx = ctypes.c_float(float(max_norm)).value
+        if not mx > 0:
+            raise ValueError("max_norm must be > 0")
+        dev = self.grad.device
+        with self._on_stream():
+            self._reduce_scatter()
+            part = torch.zeros(1, dtype=torch.float64, device=dev)
+            self.local.grad_norm(gs, part)
+            sq = torch.tensor([part.item() ** 2], dtype=torch.float64, device=dev)
+            dist.all_reduce(sq, group=self.group)
+            norm = math.sqrt(sq.item())
+            coef = mx / (norm + 1e-6)
+            self.local.step(hp, gs if coef >= 1.0 else gs * coef)   # rounded to float by the binding
+        return norm, self.all_gather_params(async_op=async_op)
+
     def step(self, hp, grad_scale=None, async_op=False):
         """Reduce-scatter (sum) the gradient bucket into this rank's slice,
         step the slice with grad_scale (default 1/world: the mean), then
         all-gather the bf16 slices.  Returns the all-gather's work handle
         when async_op is set."""
-        import torch.distributed as dist
         gs = 1.0 / self.world if grad_scale is None else float(grad_scale)
         with self._on_stream():
-            dist.reduce_scatter_tensor(self.local.array(DBUF_GRAD_BF16), self.grad, group=self.group)
+            self._reduce_scatter()
             self.local.step(hp, gs)
         return self.all_gather_params(async_op=async_op)

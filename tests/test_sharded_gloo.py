@@ -5,7 +5,9 @@ sum) into its slice -> step of the slice alone -> all-gather of the bf16
 slices.  The slice bucket is stepped by the oracle here (there is no GPU),
 so this checks the collective plumbing and the per-rank layout around the
 step: every rank must end with the whole-bucket oracle step's bf16 bucket,
-and rank r with slice r of its master weights, codes and scales.
+and rank r with slice r of its master weights, codes and scales.  The
+clipped step (step_clipped: slice norms, all-reduce of their squares) must
+give the whole bucket's norm and its clipped step.
 
 Gradients are small multiples of 2^-8 (at most 64 in size), so their sum
 over up to four ranks is exact in bf16 whatever order the reduction takes.
@@ -81,8 +83,12 @@ class OracleSlice:
     def step(self, hp, grad_scale):
         self.b.step(hp, hp["step"], grad_scale)
 
+    def grad_norm(self, grad_scale, out):
+        import oracle
+        out[0] = oracle.grad_norm(self.b.g, grad_scale)
 
-def _worker(rank, world, port, case, outdir):
+
+def _worker(rank, world, port, case, outdir, max_norm=None):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
@@ -99,13 +105,18 @@ def _worker(rank, world, port, case, outdir):
         full = _master(rows, cols)
         for i, a, b, v in sb.local_views(rb.DBUF_MASTER_F32):
             v.copy_(torch.from_numpy(full[i][a:b]))
+        norms = []
         for t in range(1, STEPS + 1):
             for g, x in zip(sb.grad_views(), _grad(rows, cols, rank, t)):
                 g.copy_(torch.from_numpy(x))
-            work = sb.step(_hp(t), async_op=(t == STEPS))
+            if max_norm is None:
+                work = sb.step(_hp(t), async_op=(t == STEPS))
+            else:
+                norm, work = sb.step_clipped(_hp(t), max_norm, async_op=(t == STEPS))
+                norms.append(norm)
             if work is not None:
                 work.wait()
-        np.savez(os.path.join(outdir, f"rank{rank}.npz"), param=sb.param.view(torch.int16).numpy(),
+        np.savez(os.path.join(outdir, f"rank{rank}.npz"), param=sb.param.view(torch.int16).numpy(), norms=norms,
                  p=local.b.p, mq=local.b.mq, vq=local.b.vq, sm=local.b.scale_m, sv=local.b.scale_v,
                  first_block=sb.rank_plan.first_block, n=sb.rank_plan.n)
         dist.barrier()
@@ -113,23 +124,34 @@ def _worker(rank, world, port, case, outdir):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("case,world", [("tiny", 2), ("tiny", 4), ("tiles", 2), ("tiles", 4), ("empty", 4)])
-def test_sharded_step_equals_the_whole_bucket(case, world, tmp_path):
+@pytest.mark.parametrize("case,world,max_norm", [("tiny", 2, None), ("tiny", 4, None), ("tiles", 2, None),
+                                                  ("tiles", 4, None), ("empty", 4, None), ("tiny", 4, 1.0),
+                                                  ("tiles", 2, 1e3)])
+def test_sharded_step_equals_the_whole_bucket(case, world, max_norm, tmp_path):
+    """max_norm set: the clipped step (global norm over all ranks' slices);
+    1.0 clips every step, 1e3 none."""
     import oracle
 
-    mp.start_processes(_worker, args=(world, _free_port(), case, str(tmp_path)), nprocs=world, join=True,
-                       start_method="spawn")
+    mp.start_processes(_worker, args=(world, _free_port(), case, str(tmp_path), max_norm), nprocs=world,
+                       join=True, start_method="spawn")
     rows, cols, k, bc = CASES[case]
     st, off, s = oracle.plan(rows, cols, k, world, 16)
     assert st == 0
     W = oracle.Bucket(rows, cols, k, off, s, world, block_cols=bc)
     for i, x in enumerate(_master(rows, cols)):
         W.p[W.tensor_slice(i)] = x.ravel()
+    want_norms = []
     for t in range(1, STEPS + 1):
         per_rank = [_grad(rows, cols, r, t) for r in range(world)]
         for i in range(len(rows)):
             W.g[W.tensor_slice(i)] = _bf16_bits(sum(g[i] for g in per_rank).ravel())
-        W.step(_hp(t), t, 1.0 / world)
+        gs = 1.0 / world
+        if max_norm is not None:
+            norm = oracle.grad_norm(W.g, gs)
+            want_norms.append(norm)
+            gs = oracle.clipped_scale(norm, gs, max_norm)
+            assert (gs < np.float32(1.0 / world)) == (max_norm == 1.0)
+        W.step(_hp(t), t, gs)
     parts = 0
     for r in range(world):
         got = np.load(tmp_path / f"rank{r}.npz")
@@ -140,6 +162,8 @@ def test_sharded_step_equals_the_whole_bucket(case, world, tmp_path):
         fb, nb = int(got["first_block"]), got["sm"].size
         assert np.array_equal(got["sm"], W.scale_m[fb:fb + nb]) and np.array_equal(got["sv"], W.scale_v[fb:fb + nb])
         parts += int(got["n"])
+        if max_norm is not None:
+            np.testing.assert_allclose(got["norms"], want_norms, rtol=1e-13)
     assert parts >= len(rows)
     if case == "empty":
         assert any(int(np.load(tmp_path / f"rank{r}.npz")["n"]) == 0 for r in range(world))
