@@ -1,5 +1,6 @@
 /* The C-ABI used from plain C99 (no C++, no CUDA headers): the host-only
- * entry points on the tiny bucket.  Built and run by tests/test_c_abi.py,
+ * entry points on the tiny bucket (planner, shards, rank buckets, work table,
+ * row-wise layout, error path).  Built and run by tests/test_c_abi.py,
  * which checks the printed numbers against the Python binding. */
 #include <stdio.h>
 #include <stdlib.h>
@@ -36,6 +37,21 @@ int main(void) {
     int64_t chunk = 0, q[3], off[3];
     if (dbuf_rowwise_layout(t, 3, 4, &chunk, q, off) != DBUF_OK) return 5;
     printf("rowwise chunk=%lld q=%lld,%lld,%lld\n", (long long)chunk, (long long)q[0], (long long)q[1], (long long)q[2]);
+    /* The RaggedShard rows of each tensor per rank, and the last rank's
+     * slice as a bucket of its own. */
+    dbuf_shard_rows shards[3 * 4];
+    if (dbuf_plan_shards(plan, shards) != DBUF_OK) return 6;
+    printf("shards_w=%lld,%lld,%lld,%lld\n", (long long)shards[0].row_end, (long long)shards[1].row_end,
+           (long long)shards[2].row_end, (long long)shards[3].row_end);
+    dbuf_plan_t* last = NULL;
+    int64_t first_block = -1, r_padding = 0, r_blocks = 0;
+    if (dbuf_plan_rank(plan, 3, &last, &first_block) != DBUF_OK) return 7;
+    if (dbuf_plan_info(last, NULL, NULL, &r_padding, &r_blocks, NULL) != DBUF_OK) return 8;
+    printf("rank3 first_block=%lld padding=%lld n_blocks=%lld\n", (long long)first_block, (long long)r_padding,
+           (long long)r_blocks);
+    dbuf_plan_t* none = NULL;
+    printf("rank_bad=%d null_out=%d\n", (int)dbuf_plan_rank(plan, 4, &none, NULL), none == NULL);
+    dbuf_plan_free(last);
     dbuf_plan_free(plan);
     dbuf_plan_free(NULL);
     return 0;

@@ -1,6 +1,6 @@
 """The C-ABI from plain C99: tests/c_abi_check.c includes only include/dbuf.h,
-links libdbuf.so, and calls the host-only entry points (planner, work
-table, required bytes, row-wise layout, error path).  Its numbers must
+links libdbuf.so, and calls the host-only entry points (planner, shards,
+rank buckets, work table, required bytes, row-wise layout, error path).  Its numbers must
 equal what the Python binding reports (CPU only)."""
 import os
 import re
@@ -35,6 +35,12 @@ def test_c99_caller(tmp_path):
     assert re.search(r"bad=%d msg_nonempty=1" % rb.DBUF_EINVAL, out.stdout), out.stdout
     chunk, q, _ = rb.dbuf_rowwise_layout(r, c, 4)
     assert f"rowwise chunk={chunk} q={q[0]},{q[1]},{q[2]}" in out.stdout
+    ends = [b for a, b in rb.dbuf_plan_shards(p, w.m)[0]]
+    assert "shards_w=" + ",".join(map(str, ends)) in out.stdout, out.stdout
+    R = rb.dbuf_plan_rank(p, 3)
+    ri = rb.dbuf_plan_info(R)
+    assert f"rank3 first_block={R.first_block} padding={ri['padding']} n_blocks={ri['n_blocks']}" in out.stdout
+    assert f"rank_bad={rb.DBUF_EINVAL} null_out=1" in out.stdout, out.stdout
 
 
 import pytest  # noqa: E402
