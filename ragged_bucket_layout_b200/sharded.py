@@ -16,12 +16,16 @@ The collectives are torch.distributed's (NCCL between GPUs), issued on the
 slice bucket's stream; the step is the library's fused kernel.  With
 async_op the all-gather is left in flight, so the next bucket's
 reduce-scatter and step can be queued behind it.
+
+ShardedMuon is the same flow for a bucket of 2-D matrices planned with one
+block per matrix: each matrix then lies whole in one slice, and its rank
+runs the library's Muon step on it.
 """
 import contextlib
 import ctypes
 import math
 
-from . import (DBUF_GRAD_BF16, DBUF_PARAM_BF16, DBuffer, dbuf_plan_info, dbuf_plan_rank)
+from . import (DBUF_GRAD_BF16, DBUF_PARAM_BF16, DBuffer, Muon, dbuf_plan_info, dbuf_plan_rank)
 
 
 class ShardedBucket:
@@ -109,7 +113,7 @@ class ShardedBucket:
             dist.all_reduce(sq, group=self.group)
             norm = math.sqrt(sq.item())
             coef = mx / (norm + 1e-6)
-            self.local.step(hp, gs if coef >= 1.0 else gs * coef)   # rounded to float by the binding
+            self._local_step(hp, gs if coef >= 1.0 else gs * coef)   # rounded to float by the binding
         return norm, self.all_gather_params(async_op=async_op)
 
     def step(self, hp, grad_scale=None, async_op=False):
@@ -120,5 +124,40 @@ class ShardedBucket:
         gs = 1.0 / self.world if grad_scale is None else float(grad_scale)
         with self._on_stream():
             self._reduce_scatter()
-            self.local.step(hp, gs)
+            self._local_step(hp, gs)
         return self.all_gather_params(async_op=async_op)
+
+    def _local_step(self, hp, grad_scale):
+        self.local.step(hp, grad_scale)
+
+
+class ShardedMuon(ShardedBucket):
+    """Distributed Muon over a bucket in which every tensor is one block
+    (planned with k = rows).  The planner then keeps each matrix whole inside
+    one slice, so the bucket's reduce-scatter delivers each matrix's summed
+    gradient to a single rank: the redistribution of a full 2-D matrix to a
+    root rank that the pages' distributed Muon does (8-bit Adam and
+    distributed Muon case study, paper Sec. 6.3).  That rank runs the
+    library's Muon step on it (momentum, Newton-Schulz on tensor cores,
+    update), and the all-gather brings the bf16 matrices back to every
+    rank.  The momentum of a matrix lives only on its rank.  `muon`
+    replaces the library's Muon state (as `local` replaces the slice
+    bucket) with any object that has step(hp, grad_scale).  hp takes the
+    keys of MUON_DEFAULTS."""
+
+    def __init__(self, plan, rank=None, world=None, group=None, device="cuda", local=None, muon=None):
+        super().__init__(plan, rank, world, group, device, local)
+        for i, a, b in self.rank_plan.parts:
+            if a != 0 or b != plan.shapes[i][0]:
+                raise ValueError(f"tensor {i} is split between ranks: plan a Muon bucket with k = rows")
+        self.matrices = [i for i, _, _ in self.rank_plan.parts]   # the tensors this rank steps
+        if muon is not None:
+            self.muon = muon
+        else:
+            # dbuf_muon_create needs at least one tensor; a rank without any
+            # has only padding, which stays zero.
+            self.muon = Muon(self.local, range(self.rank_plan.n)) if self.rank_plan.n else None
+
+    def _local_step(self, hp, grad_scale):
+        if self.muon is not None:
+            self.muon.step(hp, grad_scale)

@@ -13,7 +13,7 @@ import torch
 import ragged_bucket_layout_b200 as rb
 import synth
 
-from test_rank_buckets import EDGE_CASES, _case
+from test_oracle_rank_buckets import EDGE_CASES, _case
 
 pytestmark = pytest.mark.gpu
 

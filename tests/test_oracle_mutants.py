@@ -88,6 +88,16 @@ PY_MUTANTS = {
                               "test_oracle_muon.py::test_momentum_of_a_constant_gradient"),
     "momentum_unscaled": ("    t = g * np.float32(grad_scale)", "    t = g",
                           "test_oracle_muon.py::test_momentum_of_a_constant_gradient"),
+    "rank_not_rebased": ('        out["offsets"].append(a - lo)', '        out["offsets"].append(a - o)',
+                         "test_oracle_rank_buckets.py::test_rank_buckets_step_like_the_whole_bucket"),
+    "rank_first_block_floor": ("        first_block += tiles_per_row_block * (-(-first_row_in // K))",
+                               "        first_block += tiles_per_row_block * (first_row_in // K)",
+                               "test_oracle_rank_buckets.py::test_rank_buckets_step_like_the_whole_bucket"),
+    "rank_first_block_rows_only": ("        first_block += tiles_per_row_block * (-(-first_row_in // K))",
+                                   "        first_block += -(-first_row_in // K)",
+                                   "test_oracle_rank_buckets.py::test_first_block_counts_the_blocks_before_the_slice"),
+    "rank_tiles_dropped": ('        out["block_cols"].append(int(bc[i]))', '        out["block_cols"].append(0)',
+                           "test_oracle_rank_buckets.py::test_rank_buckets_step_like_the_whole_bucket"),
     "rowwise_unscaled": ("            pack(g[r0 * int(cols[t]):r0 * int(cols[t]) + k], seg, scale)",
                          "            pack(g[r0 * int(cols[t]):r0 * int(cols[t]) + k], seg, 1.0)",
                          "test_oracle_rowwise.py::test_golden_rowwise_layout"),
@@ -112,7 +122,7 @@ def test_pin_catches_planted_mistake(name, tmp_path):
     shutil.copytree(os.path.join(ROOT, "synth"), work / "synth",
                     ignore=shutil.ignore_patterns("__pycache__"))
     for f in ("conftest.py", "test_oracle_adam.py", "test_oracle_layout.py", "test_oracle_rowwise.py",
-              "test_oracle_tiles.py", "test_oracle_muon.py"):
+              "test_oracle_tiles.py", "test_oracle_muon.py", "test_oracle_rank_buckets.py"):
         shutil.copy(os.path.join(ROOT, "tests", f), work / "tests" / f)
     shutil.copytree(os.path.join(ROOT, "tests", "golden"), work / "tests" / "golden")
     (work / "oracle" / fname).write_text(src.replace(orig, bad))

@@ -167,3 +167,123 @@ def test_sharded_step_equals_the_whole_bucket(case, world, max_norm, tmp_path):
     assert parts >= len(rows)
     if case == "empty":
         assert any(int(np.load(tmp_path / f"rank{r}.npz")["n"]) == 0 for r in range(world))
+
+
+# ------------------------------------------------------------ distributed Muon
+
+MUON_CASES = {
+    # rows, cols of 2-D matrices (a tall one, a wide one); each is one block
+    "mats": ([64, 48, 96, 32, 40], [32, 64, 16, 32, 24]),
+    # two matrices for four ranks: two ranks hold none
+    "few": ([128, 16], [64, 16]),
+}
+MUON_HP = dict(lr=0.02, momentum=0.95, weight_decay=0.01, eps=1e-7, ns_steps=5, nesterov=1)
+
+
+def _muon_matrix_step(p, pb, g_bits, mom, R, C, hp, gs):
+    """One Muon step of one matrix from the oracle's pieces, in place on the
+    fp32 master p, its bf16 copy pb and the momentum (flat views)."""
+    import oracle
+    U = oracle.muon_momentum(mom, g_bits, hp["momentum"], gs, nesterov=True)
+    X = oracle.newton_schulz(U.reshape(R, C).astype(np.float64), hp["ns_steps"], hp["eps"])
+    lrs = np.float32(hp["lr"] * oracle.muon_update_scale(R, C))
+    decay = np.float32(1.0 - hp["lr"] * hp["weight_decay"])
+    p[:] = p * decay - lrs * X.astype(np.float32).ravel()
+    pb[:] = oracle.bf16_round(p)
+
+
+class OracleMuon:
+    """Muon state of the matrices in one rank's slice bucket, stepped with
+    the oracle's pieces."""
+
+    def __init__(self, local):
+        self.local = local
+        rk = local.rk
+        self.mats = [(int(o), int(r), int(c)) for r, c, o in zip(rk["rows"], rk["cols"], rk["offsets"])]
+        self.mom = [np.zeros(r * c, np.float32) for _, r, c in self.mats]
+
+    def step(self, hp, grad_scale):
+        b = self.local.b
+        for (o, R, C), mom in zip(self.mats, self.mom):
+            sl = slice(o, o + R * C)
+            _muon_matrix_step(b.p[sl], b.pb[sl], b.g[sl], mom, R, C, hp, grad_scale)
+
+
+def _muon_worker(rank, world, port, case, outdir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        import oracle
+        import ragged_bucket_layout_b200 as rb
+        from ragged_bucket_layout_b200.sharded import ShardedMuon
+
+        rows, cols = MUON_CASES[case]
+        plan = rb.dbuf_plan(rows, cols, rows, world, 16)            # k = rows: one block per matrix
+        info = rb.dbuf_plan_info(plan)
+        local = OracleSlice(oracle.rank_bucket(rows, cols, rows, info["offsets"], info["slice"], world, rank))
+        sm = ShardedMuon(plan, local=local, muon=OracleMuon(local))
+        full = _master(rows, cols)
+        for i, a, b, v in sm.local_views(rb.DBUF_MASTER_F32):
+            assert (a, b) == (0, rows[i])                          # whole matrices only
+            v.copy_(torch.from_numpy(full[i]))
+        for t in range(1, STEPS + 1):
+            for g, x in zip(sm.grad_views(), _grad(rows, cols, rank, t)):
+                g.copy_(torch.from_numpy(x))
+            sm.step(MUON_HP)
+        np.savez(os.path.join(outdir, f"rank{rank}.npz"), param=sm.param.view(torch.int16).numpy(), p=local.b.p,
+                 mats=np.array(sm.matrices, np.int64), mom=np.concatenate([np.zeros(0, np.float32)] + sm.muon.mom))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("case,world", [("mats", 2), ("mats", 4), ("few", 4)])
+def test_sharded_muon_steps_every_matrix_once_on_its_rank(case, world, tmp_path):
+    import oracle
+
+    mp.start_processes(_muon_worker, args=(world, _free_port(), case, str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    rows, cols = MUON_CASES[case]
+    st, off, s = oracle.plan(rows, cols, rows, world, 16)
+    assert st == 0
+    W = oracle.Bucket(rows, cols, rows, off, s, world)
+    moms = [np.zeros(r * c, np.float32) for r, c in zip(rows, cols)]
+    for i, x in enumerate(_master(rows, cols)):
+        W.p[W.tensor_slice(i)] = x.ravel()
+    for t in range(1, STEPS + 1):
+        per_rank = [_grad(rows, cols, r, t) for r in range(world)]
+        for i in range(len(rows)):
+            sl = W.tensor_slice(i)
+            W.g[sl] = _bf16_bits(sum(g[i] for g in per_rank).ravel())
+            _muon_matrix_step(W.p[sl], W.pb[sl], W.g[sl], moms[i], rows[i], cols[i], MUON_HP, 1.0 / world)
+    owners = []
+    for r in range(world):
+        got = np.load(tmp_path / f"rank{r}.npz")
+        assert np.array_equal(got["param"].view(np.uint16), W.pb), f"rank {r}: gathered bf16 bucket"
+        assert np.array_equal(got["p"].view(np.uint32), W.p[r * s:(r + 1) * s].view(np.uint32)), f"rank {r}"
+        mats = got["mats"].tolist()
+        want_mom = np.concatenate([np.zeros(0, np.float32)] + [moms[i] for i in mats])
+        assert np.array_equal(got["mom"], want_mom), f"rank {r}: momentum"
+        owners += mats
+    assert sorted(owners) == list(range(len(rows)))               # every matrix on exactly one rank
+    assert len(set(owners)) == len(rows) and world > 1
+
+
+def test_sharded_muon_refuses_a_split_matrix():
+    """With blocks of fewer rows than the matrix, a slice boundary can cut a
+    matrix; Muon needs it whole on one rank, so the plan is refused."""
+    import oracle
+    import ragged_bucket_layout_b200 as rb
+    from ragged_bucket_layout_b200.sharded import ShardedMuon
+
+    rows, cols = [64, 64], [32, 32]
+    plan = rb.dbuf_plan(rows, cols, [8, 8], 4, 16)
+    info = rb.dbuf_plan_info(plan)
+    assert any(a > 0 for q in range(4) for _, a, _ in rb.dbuf_plan_rank(plan, q).parts)
+    for q in range(4):
+        local = OracleSlice(oracle.rank_bucket(rows, cols, [8, 8], info["offsets"], info["slice"], 4, q))
+        parts = rb.dbuf_plan_rank(plan, q).parts
+        if all(a == 0 and b == rows[i] for i, a, b in parts):
+            continue
+        with pytest.raises(ValueError, match="k = rows"):
+            ShardedMuon(plan, rank=q, world=4, local=local, muon=object())
