@@ -427,12 +427,33 @@ class DBuffer:
     C-ABI calls above on the given (or current) CUDA stream.
     """
 
-    def __init__(self, plan, device="cuda", stream=None):
+    def __init__(self, plan, device="cuda", stream=None, alloc=None):
+        """alloc: optional allocation hook, called once as alloc(nbytes).  It
+        returns a contiguous 1-D uint8 tensor of at least nbytes on the
+        device, 256-byte aligned (e.g. a slice of the caller's memory pool),
+        and the bucket lives there.  A hook that returns None or raises
+        MemoryError gives DbufError(DBUF_ENOMEM), before any device work;
+        so does running out of memory on the default path."""
         import torch
         self.plan = plan
         self.info = dbuf_plan_info(plan)
-        nbytes = dbuf_required_bytes(plan)
-        self.base = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+        nbytes = max(dbuf_required_bytes(plan), 256)
+        if alloc is None:
+            try:
+                base = torch.empty(nbytes, dtype=torch.uint8, device=device)
+            except torch.OutOfMemoryError as e:
+                raise DbufError(DBUF_ENOMEM, f"allocating {nbytes} bytes: {e}") from e
+        else:
+            try:
+                base = alloc(nbytes)
+            except MemoryError as e:
+                raise DbufError(DBUF_ENOMEM, f"allocation hook failed for {nbytes} bytes: {e}") from e
+            if base is None:
+                raise DbufError(DBUF_ENOMEM, f"allocation hook returned no memory for {nbytes} bytes")
+            if not isinstance(base, torch.Tensor) or base.dtype != torch.uint8 or base.dim() != 1 \
+                    or not base.is_contiguous():
+                raise DbufError(DBUF_EINVAL, "allocation hook must return a contiguous 1-D uint8 tensor")
+        self.base = base
         self.stream = stream if stream is not None else torch.cuda.current_stream(self.base.device)
         self._destroy = _lib.dbuf_destroy   # held here: module globals may be gone at interpreter exit
         self.handle = dbuf_create(plan, self.base.data_ptr(), self.base.numel(), self.stream)

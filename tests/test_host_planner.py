@@ -13,6 +13,7 @@ import subprocess
 
 import numpy as np
 import pytest
+import torch
 
 import oracle
 import ragged_bucket_layout_b200 as rb
@@ -324,3 +325,27 @@ def test_oracle_shards_against_per_element_slices():
         e = int(off[i]) + np.arange(int(r[i] * c[i]))
         counts = np.bincount(e // s, minlength=w.m)
         assert [(hi - lo) * int(c[i]) for lo, hi in sh[i]] == counts.tolist()
+
+
+def test_allocation_hook_failures_are_reported_before_device_work():
+    """DBuffer's allocation hook (the caller's memory pool): a hook that
+    fails, or returns no memory or the wrong kind of memory, is reported as a
+    DbufError before any device call, so this runs without a GPU."""
+    p = rb.dbuf_plan([64, 8], [64, 16], [4, 8], 2, 16)
+    need = max(rb.dbuf_required_bytes(p), 256)
+    asked = []
+
+    def none(n):
+        asked.append(n)
+        return None
+
+    def raises(n):
+        raise MemoryError("pool exhausted")
+
+    for hook, status in ((none, rb.DBUF_ENOMEM), (raises, rb.DBUF_ENOMEM),
+                         (lambda n: torch.empty(n, dtype=torch.float32), rb.DBUF_EINVAL),
+                         (lambda n: torch.empty((n, 2), dtype=torch.uint8), rb.DBUF_EINVAL)):
+        with pytest.raises(rb.DbufError) as e:
+            rb.DBuffer(p, alloc=hook)
+        assert e.value.status == status
+    assert asked == [need]
