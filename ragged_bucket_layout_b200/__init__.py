@@ -173,7 +173,17 @@ def dbuf_plan_rank(plan, rank):
         raise ValueError("dbuf_plan_rank needs a plan made by dbuf_plan (m unknown)")
     out, fb = ctypes.c_void_p(), ctypes.c_int64()
     _check(_lib.dbuf_plan_rank(plan.handle, int(rank), ctypes.byref(out), ctypes.byref(fb)))
-    parts = [(i, a, b) for i, per in enumerate(dbuf_plan_shards(plan, plan.m)) for a, b in [per[rank]] if b > a]
+    if getattr(plan, "shapes", None) is not None:
+        # This rank's row ranges only: O(n), not the n*m table of dbuf_plan_shards.
+        info = dbuf_plan_info(plan)
+        lo, hi = int(rank) * info["slice"], (int(rank) + 1) * info["slice"]
+        parts = []
+        for i, (o, (R, C)) in enumerate(zip(info["offsets"], plan.shapes)):
+            a, b = min(R * C, max(0, lo - o)), min(R * C, max(0, hi - o))
+            if b > a:
+                parts.append((i, a // C, b // C))
+    else:
+        parts = [(i, a, b) for i, per in enumerate(dbuf_plan_shards(plan, plan.m)) for a, b in [per[rank]] if b > a]
     sub = Plan(out.value, len(parts), 1)
     sub.rank, sub.first_block, sub.parts = int(rank), fb.value, parts
     if getattr(plan, "shapes", None) is not None:
