@@ -287,3 +287,27 @@ def test_sharded_muon_refuses_a_split_matrix():
             continue
         with pytest.raises(ValueError, match="k = rows"):
             ShardedMuon(plan, rank=q, world=4, local=local, muon=object())
+
+
+def test_sharded_bucket_checks_its_arguments():
+    """A plan for another number of ranks, or a plan that is not from
+    dbuf_plan (no tensor shapes), is refused before any collective."""
+    import oracle
+    import ragged_bucket_layout_b200 as rb
+    from ragged_bucket_layout_b200.sharded import ShardedBucket
+
+    rows, cols, k, bc = CASES["tiny"]
+    plan = rb.dbuf_plan(rows, cols, k, 4, 16)
+    info = rb.dbuf_plan_info(plan)
+    local = OracleSlice(oracle.rank_bucket(rows, cols, k, info["offsets"], info["slice"], 4, 0))
+    with pytest.raises(ValueError, match="4 slices for 2 ranks"):
+        ShardedBucket(plan, rank=0, world=2, local=local)
+    bare = rb.Plan(plan.handle, plan.n, plan.m)            # same layout, no shapes
+    try:
+        with pytest.raises(ValueError, match="dbuf_plan"):
+            ShardedBucket(bare, rank=0, world=4, local=local)
+    finally:
+        bare.handle = None                                 # owned by `plan`
+    sb = ShardedBucket(plan, rank=0, world=4, local=local)
+    assert [tuple(v.shape) for v in sb.grad_views()] == list(zip(rows, cols))
+    assert sb.grad.numel() == sb.param.numel() == info["bucket"]
