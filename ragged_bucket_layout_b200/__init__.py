@@ -157,8 +157,12 @@ def dbuf_plan_info(plan):
                 offsets=[offs[i] for i in range(plan.n)])
 
 
-def dbuf_plan_shards(plan, m):
-    """RaggedShard placement: [[(row_begin, row_end) for each rank] for each tensor]."""
+def dbuf_plan_shards(plan, m=None):
+    """RaggedShard placement: [[(row_begin, row_end) for each rank] for each
+    tensor].  m defaults to the plan's own slice count."""
+    m = plan.m if m is None else int(m)
+    if m is None or (plan.m is not None and m != plan.m):
+        raise ValueError("m must be the plan's slice count")
     arr = (ctypes.c_int64 * max(2 * plan.n * m, 1))()
     _check(_lib.dbuf_plan_shards(plan.handle, arr))
     return [[(arr[2 * (i * m + r)], arr[2 * (i * m + r) + 1]) for r in range(m)] for i in range(plan.n)]
