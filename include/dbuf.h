@@ -97,6 +97,11 @@ dbuf_status dbuf_plan_info(const dbuf_plan_t* plan, int64_t* slice_elems, int64_
 
 void dbuf_plan_free(dbuf_plan_t* plan); /* NULL is a no-op */
 
+/* Number of tensors and of slices of a plan (the sizes of the caller-owned
+ * arrays that dbuf_plan_info, dbuf_plan_shards and dbuf_unpack_views fill).
+ * Either output may be NULL.  Host only. */
+dbuf_status dbuf_plan_dims(const dbuf_plan_t* plan, int32_t* n_tensors, int32_t* m);
+
 /* RaggedShard placement of a plan (paper Sec. 3; page section
  * "1. RaggedShard": devices hold different numbers of whole blocks): the
  * rows of each tensor that each rank's slice holds.  out[i*m + r] (host

@@ -62,6 +62,7 @@ _SIGS = {
     "dbuf_plan_free": (None, [_P]),
     "dbuf_plan_shards": (ctypes.c_int, [_P, _P]),
     "dbuf_plan_rank": (ctypes.c_int, [_P, _i32, _PP, _pi64]),
+    "dbuf_plan_dims": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]),
     "dbuf_required_bytes": (_sz, [_P]),
     "dbuf_create": (ctypes.c_int, [_P, _P, _sz, _P, _PP]),
     "dbuf_pack_grads": (ctypes.c_int, [_P, _PP, _f32, _P]),
@@ -149,23 +150,25 @@ def dbuf_plan(rows, cols, k, m, align_elems=16, max_bucket_elems=0, block_cols=N
 
 
 def dbuf_plan_info(plan):
+    n = dbuf_plan_dims(plan)[0]
     s, b, p, nb = (ctypes.c_int64() for _ in range(4))
-    offs = (ctypes.c_int64 * max(plan.n, 1))()
+    offs = (ctypes.c_int64 * max(n, 1))()
     _check(_lib.dbuf_plan_info(plan.handle, ctypes.byref(s), ctypes.byref(b), ctypes.byref(p),
                                ctypes.byref(nb), offs))
     return dict(slice=s.value, bucket=b.value, padding=p.value, n_blocks=nb.value,
-                offsets=[offs[i] for i in range(plan.n)])
+                offsets=[offs[i] for i in range(n)])
 
 
 def dbuf_plan_shards(plan, m=None):
     """RaggedShard placement: [[(row_begin, row_end) for each rank] for each
     tensor].  m defaults to the plan's own slice count."""
-    m = plan.m if m is None else int(m)
-    if m is None or (plan.m is not None and m != plan.m):
-        raise ValueError("m must be the plan's slice count")
-    arr = (ctypes.c_int64 * max(2 * plan.n * m, 1))()
+    n, pm = dbuf_plan_dims(plan)
+    if m is not None and int(m) != pm:
+        raise ValueError(f"m must be the plan's slice count ({pm})")
+    m = pm
+    arr = (ctypes.c_int64 * max(2 * n * m, 1))()
     _check(_lib.dbuf_plan_shards(plan.handle, arr))
-    return [[(arr[2 * (i * m + r)], arr[2 * (i * m + r) + 1]) for r in range(m)] for i in range(plan.n)]
+    return [[(arr[2 * (i * m + r)], arr[2 * (i * m + r) + 1]) for r in range(m)] for i in range(n)]
 
 
 def dbuf_plan_rank(plan, rank):
@@ -189,10 +192,20 @@ def dbuf_plan_rank(plan, rank):
     else:
         parts = [(i, a, b) for i, per in enumerate(dbuf_plan_shards(plan, plan.m)) for a, b in [per[rank]] if b > a]
     sub = Plan(out.value, len(parts), 1)
+    if dbuf_plan_dims(sub) != (len(parts), 1):
+        raise DbufError(DBUF_EINVAL, f"rank {rank}: the library's rank plan has {dbuf_plan_dims(sub)[0]} tensors, "
+                                     f"the binding found {len(parts)}")
     sub.rank, sub.first_block, sub.parts = int(rank), fb.value, parts
     if getattr(plan, "shapes", None) is not None:
         sub.shapes = [(b - a, plan.shapes[i][1]) for i, a, b in parts]
     return sub
+
+
+def dbuf_plan_dims(plan):
+    """(number of tensors, number of slices) as the library holds them."""
+    n, m = ctypes.c_int32(), ctypes.c_int32()
+    _check(_lib.dbuf_plan_dims(plan.handle, ctypes.byref(n), ctypes.byref(m)))
+    return n.value, m.value
 
 
 def dbuf_plan_free(plan):
@@ -491,7 +504,7 @@ class DBuffer:
 
     def views(self, which):
         out = []
-        for ptr, rows, cols, _ in dbuf_unpack_views(self.handle, which, self.plan.n):
+        for ptr, rows, cols, _ in dbuf_unpack_views(self.handle, which, dbuf_plan_dims(self.plan)[0]):
             out.append(self._view(ptr, rows * cols, which).view(rows, cols))
         return out
 

@@ -211,6 +211,13 @@ extern "C" dbuf_status dbuf_plan_info(const dbuf_plan_t* plan, int64_t* slice_el
     return DBUF_OK;
 }
 
+extern "C" dbuf_status dbuf_plan_dims(const dbuf_plan_t* plan, int32_t* n_tensors, int32_t* m) {
+    if (!plan) return dbuf_detail::fail(DBUF_EINVAL, "dbuf_plan_dims: plan is NULL");
+    if (n_tensors) *n_tensors = plan->n;
+    if (m) *m = plan->m;
+    return DBUF_OK;
+}
+
 extern "C" dbuf_status dbuf_plan_shards(const dbuf_plan_t* plan, dbuf_shard_rows* out) {
     if (!plan) return dbuf_detail::fail(DBUF_EINVAL, "dbuf_plan_shards: plan is NULL");
     if (plan->n > 0 && !out) return dbuf_detail::fail(DBUF_EINVAL, "dbuf_plan_shards: out is NULL");

@@ -49,6 +49,9 @@ int main(void) {
     if (dbuf_plan_info(last, NULL, NULL, &r_padding, &r_blocks, NULL) != DBUF_OK) return 8;
     printf("rank3 first_block=%lld padding=%lld n_blocks=%lld\n", (long long)first_block, (long long)r_padding,
            (long long)r_blocks);
+    int32_t dn = -1, dm = -1, rn = -1, rm = -1;
+    if (dbuf_plan_dims(plan, &dn, &dm) != DBUF_OK || dbuf_plan_dims(last, &rn, &rm) != DBUF_OK) return 9;
+    printf("dims=%d,%d rank3_dims=%d,%d\n", (int)dn, (int)dm, (int)rn, (int)rm);
     dbuf_plan_t* none = NULL;
     printf("rank_bad=%d null_out=%d\n", (int)dbuf_plan_rank(plan, 4, &none, NULL), none == NULL);
     dbuf_plan_free(last);

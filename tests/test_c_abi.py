@@ -41,6 +41,7 @@ def test_c99_caller(tmp_path):
     ri = rb.dbuf_plan_info(R)
     assert f"rank3 first_block={R.first_block} padding={ri['padding']} n_blocks={ri['n_blocks']}" in out.stdout
     assert f"rank_bad={rb.DBUF_EINVAL} null_out=1" in out.stdout, out.stdout
+    assert f"dims=3,4 rank3_dims={R.n},1" in out.stdout, out.stdout
 
 
 import pytest  # noqa: E402

@@ -104,12 +104,13 @@ def test_plan_rank_errors_and_identity():
 @pytest.mark.parametrize("name", ["tiny_m4", "tiles_cut_m4", "empty_slices_m4", "moe_layer_m64"])
 def test_rank_parts_agree_with_the_shard_table(name):
     """The binding's per-rank part list (from offsets and shapes) equals the
-    rows dbuf_plan_shards gives for that rank, and the library's rank plan
-    puts each part at its parent offset minus q*s."""
+    rows dbuf_plan_shards gives for that rank; the library's rank plan holds
+    as many tensors and puts each at its parent offset minus q*s."""
     r, c, k, bc, m, align, P, off, s = _plans(name)
     table = rb.dbuf_plan_shards(P, m)
     for q in range(m):
         R = rb.dbuf_plan_rank(P, q)
         assert R.parts == [(i, a, b) for i, per in enumerate(table) for a, b in [per[q]] if b > a]
+        assert rb.dbuf_plan_dims(R) == (len(R.parts), 1)
         want = [int(off[i]) + a * int(c[i]) - q * s for i, a, b in R.parts]
         assert rb.dbuf_plan_info(R)["offsets"] == want
