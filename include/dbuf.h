@@ -19,6 +19,9 @@
  *     per tensor; streams are ordered explicitly (no record_stream).
  *   8-bit Adam case study (paper Sec. 6.3): block-wise quantised optimizer
  *     states, each device quantising its own blocks with no communication.
+ *     A dbuf holds all m slices of a bucket (m devices simulated on one), or,
+ *     from dbuf_plan_rank, a single device's slice with only that slice's
+ *     optimizer state.
  *
  * Conventions of every entry point:
  *   - Status codes are returned; on failure dbuf_last_error() gives a
