@@ -301,7 +301,9 @@ def run_ours(args):
 
     w = synth.workload(args.workload)
     r, c, k = w.arrays()
+    t_plan = time.perf_counter()
     plan = rb.dbuf_plan(r, c, k, w.m, w.align)
+    planner_ms = (time.perf_counter() - t_plan) * 1e3       # host, once at init
     info = rb.dbuf_plan_info(plan)
     stats = workload_stats(w, info)
     stream = torch.cuda.Stream()
@@ -538,7 +540,8 @@ def run_ours(args):
         "warmup": args.warmup, "ms_per_step": per_step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": w.name, "params": stats["params"], "blocks": stats["blocks"],
-                   "padding": stats["padding"], "bucket_elems": stats["bucket"], "m": w.m,
+                   "padding": stats["padding"], "padding_frac": stats["padding"] / stats["bucket"],
+                   "planner_ms": planner_ms, "bucket_elems": stats["bucket"], "m": w.m,
                    "bytes_per_step": stats["step_bytes"],
                    "l2": f"inputs larger than L2 ({stats['step_bytes'] / 1e9:.2f} GB moved per step)",
                    "parallelism": f"dp{world} (one bucket per rank, no data-path collective)"},
