@@ -311,3 +311,65 @@ def test_sharded_bucket_checks_its_arguments():
     sb = ShardedBucket(plan, rank=0, world=4, local=local)
     assert [tuple(v.shape) for v in sb.grad_views()] == list(zip(rows, cols))
     assert sb.grad.numel() == sb.param.numel() == info["bucket"]
+
+
+def _multi_worker(rank, world, port, outdir):
+    """Two buckets stepped back to back, each all-gather left in flight while
+    the next bucket's reduce-scatter and step run (the overlap pattern)."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        import oracle
+        import ragged_bucket_layout_b200 as rb
+        from ragged_bucket_layout_b200.sharded import ShardedBucket
+
+        sbs, locals_ = [], []
+        for case in ("tiny", "tiles"):
+            rows, cols, k, bc = CASES[case]
+            plan = rb.dbuf_plan(rows, cols, k, world, 16, block_cols=bc)
+            info = rb.dbuf_plan_info(plan)
+            local = OracleSlice(oracle.rank_bucket(rows, cols, k, info["offsets"], info["slice"], world, rank, bc))
+            sb = ShardedBucket(plan, local=local)
+            full = _master(rows, cols)
+            for i, a, b, v in sb.local_views(rb.DBUF_MASTER_F32):
+                v.copy_(torch.from_numpy(full[i][a:b]))
+            sbs.append(sb)
+            locals_.append(local)
+        for t in range(1, STEPS + 1):
+            works = []
+            for sb, case in zip(sbs, ("tiny", "tiles")):
+                rows, cols, _, _ = CASES[case]
+                for g, x in zip(sb.grad_views(), _grad(rows, cols, rank, t)):
+                    g.copy_(torch.from_numpy(x))
+                works.append(sb.step(_hp(t), async_op=True))
+            for w in works:
+                w.wait()
+        for j, (sb, local) in enumerate(zip(sbs, locals_)):
+            np.savez(os.path.join(outdir, f"rank{rank}_b{j}.npz"), param=sb.param.view(torch.int16).numpy(),
+                     p=local.b.p)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_buckets_with_all_gathers_in_flight(tmp_path):
+    import oracle
+
+    world = 2
+    mp.start_processes(_multi_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    for j, case in enumerate(("tiny", "tiles")):
+        rows, cols, k, bc = CASES[case]
+        st, off, s = oracle.plan(rows, cols, k, world, 16)
+        W = oracle.Bucket(rows, cols, k, off, s, world, block_cols=bc)
+        for i, x in enumerate(_master(rows, cols)):
+            W.p[W.tensor_slice(i)] = x.ravel()
+        for t in range(1, STEPS + 1):
+            per_rank = [_grad(rows, cols, r, t) for r in range(world)]
+            for i in range(len(rows)):
+                W.g[W.tensor_slice(i)] = _bf16_bits(sum(g[i] for g in per_rank).ravel())
+            W.step(_hp(t), t, 1.0 / world)
+        for r in range(world):
+            got = np.load(tmp_path / f"rank{r}_b{j}.npz")
+            assert np.array_equal(got["param"].view(np.uint16), W.pb), f"bucket {case}, rank {r}"
+            assert np.array_equal(got["p"].view(np.uint32), W.p[r * s:(r + 1) * s].view(np.uint32))
