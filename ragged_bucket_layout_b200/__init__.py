@@ -146,6 +146,9 @@ def dbuf_plan(rows, cols, k, m, align_elems=16, max_bucket_elems=0, block_cols=N
     _check(_lib.dbuf_plan(descs, n, int(m), int(align_elems), int(max_bucket_elems), ctypes.byref(out)))
     plan = Plan(out.value, n, int(m))
     plan.shapes = [(int(r), int(c)) for r, c in zip(rows, cols)]
+    plan.k = [int(q) for q in k]
+    plan.block_cols = bc
+    plan.align = int(align_elems)
     return plan
 
 

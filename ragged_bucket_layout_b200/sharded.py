@@ -23,6 +23,7 @@ runs the library's Muon step on it.
 """
 import contextlib
 import ctypes
+import hashlib
 import math
 
 from . import (DBUF_GRAD_BF16, DBUF_PARAM_BF16, DBuffer, Muon, dbuf_plan_info, dbuf_plan_rank)
@@ -35,7 +36,9 @@ class ShardedBucket:
     has array(which), views(which) and step(hp, grad_scale), e.g. a host-side
     model of it."""
 
-    def __init__(self, plan, rank=None, world=None, group=None, device="cuda", local=None):
+    def __init__(self, plan, rank=None, world=None, group=None, device="cuda", local=None, check_plan=True):
+        """check_plan: compare a digest of the plan across the group first
+        (one all_gather_object), and raise on every rank if they differ."""
         import torch
         import torch.distributed as dist
 
@@ -46,15 +49,32 @@ class ShardedBucket:
             raise ValueError(f"the plan has {plan.m} slices for {self.world} ranks")
         if getattr(plan, "shapes", None) is None:
             raise ValueError("ShardedBucket needs a plan made by dbuf_plan")
+        info = dbuf_plan_info(plan)
+        if check_plan and self.world > 1:
+            self._check_same_plan(plan, info)
         self.plan = plan
         self.rank_plan = dbuf_plan_rank(plan, self.rank)
-        info = dbuf_plan_info(plan)
         self.slice, self.offsets = info["slice"], info["offsets"]
         self.local = DBuffer(self.rank_plan, device=device) if local is None else local
         dev = self.local.array(DBUF_GRAD_BF16).device
         with self._on_stream():
             self.grad = torch.zeros(info["bucket"], dtype=torch.bfloat16, device=dev)
             self.param = torch.zeros(info["bucket"], dtype=torch.bfloat16, device=dev)
+
+    def _check_same_plan(self, plan, info):
+        """Every rank plans its bucket on its own; if the ranks' tensor lists
+        differ (another order, another shape), the collectives would mix
+        unrelated data.  Compare digests of the plans and fail loudly."""
+        import torch.distributed as dist
+        desc = repr((plan.shapes, getattr(plan, "k", None), getattr(plan, "block_cols", None),
+                     info["slice"], info["offsets"], plan.m))
+        mine = hashlib.sha256(desc.encode()).hexdigest()
+        digests = [None] * self.world
+        dist.all_gather_object(digests, mine, group=self.group)
+        bad = [r for r, d in enumerate(digests) if d != digests[0]]
+        if bad:
+            raise RuntimeError(f"ranks disagree on the bucket plan (ranks {bad} differ from rank 0); "
+                               "every rank must pass the same tensors in the same order")
 
     def _on_stream(self):
         import torch
@@ -145,8 +165,9 @@ class ShardedMuon(ShardedBucket):
     bucket) with any object that has step(hp, grad_scale).  hp takes the
     keys of MUON_DEFAULTS."""
 
-    def __init__(self, plan, rank=None, world=None, group=None, device="cuda", local=None, muon=None):
-        super().__init__(plan, rank, world, group, device, local)
+    def __init__(self, plan, rank=None, world=None, group=None, device="cuda", local=None, muon=None,
+                 check_plan=True):
+        super().__init__(plan, rank, world, group, device, local, check_plan)
         for i, a, b in self.rank_plan.parts:
             if a != 0 or b != plan.shapes[i][0]:
                 raise ValueError(f"tensor {i} is split between ranks: plan a Muon bucket with k = rows")

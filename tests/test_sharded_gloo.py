@@ -286,7 +286,7 @@ def test_sharded_muon_refuses_a_split_matrix():
         if all(a == 0 and b == rows[i] for i, a, b in parts):
             continue
         with pytest.raises(ValueError, match="k = rows"):
-            ShardedMuon(plan, rank=q, world=4, local=local, muon=object())
+            ShardedMuon(plan, rank=q, world=4, local=local, muon=object(), check_plan=False)
 
 
 def test_sharded_bucket_checks_its_arguments():
@@ -301,14 +301,14 @@ def test_sharded_bucket_checks_its_arguments():
     info = rb.dbuf_plan_info(plan)
     local = OracleSlice(oracle.rank_bucket(rows, cols, k, info["offsets"], info["slice"], 4, 0))
     with pytest.raises(ValueError, match="4 slices for 2 ranks"):
-        ShardedBucket(plan, rank=0, world=2, local=local)
+        ShardedBucket(plan, rank=0, world=2, local=local, check_plan=False)
     bare = rb.Plan(plan.handle, plan.n, plan.m)            # same layout, no shapes
     try:
         with pytest.raises(ValueError, match="dbuf_plan"):
-            ShardedBucket(bare, rank=0, world=4, local=local)
+            ShardedBucket(bare, rank=0, world=4, local=local, check_plan=False)
     finally:
         bare.handle = None                                 # owned by `plan`
-    sb = ShardedBucket(plan, rank=0, world=4, local=local)
+    sb = ShardedBucket(plan, rank=0, world=4, local=local, check_plan=False)
     assert [tuple(v.shape) for v in sb.grad_views()] == list(zip(rows, cols))
     assert sb.grad.numel() == sb.param.numel() == info["bucket"]
 
@@ -373,3 +373,40 @@ def test_two_buckets_with_all_gathers_in_flight(tmp_path):
             got = np.load(tmp_path / f"rank{r}_b{j}.npz")
             assert np.array_equal(got["param"].view(np.uint16), W.pb), f"bucket {case}, rank {r}"
             assert np.array_equal(got["p"].view(np.uint32), W.p[r * s:(r + 1) * s].view(np.uint32))
+
+
+def _disagree_worker(rank, world, port, outdir):
+    """Rank 1 lists the same tensors in another order: every rank must get
+    an error at construction, before any reduce-scatter."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        import oracle
+        import ragged_bucket_layout_b200 as rb
+        from ragged_bucket_layout_b200.sharded import ShardedBucket
+
+        rows, cols, k, bc = CASES["tiles"]
+        if rank == 1:
+            rows, cols, k, bc = rows[::-1], cols[::-1], k[::-1], bc[::-1]
+        plan = rb.dbuf_plan(rows, cols, k, world, 16, block_cols=bc)
+        info = rb.dbuf_plan_info(plan)
+        local = OracleSlice(oracle.rank_bucket(rows, cols, k, info["offsets"], info["slice"], world, rank, bc))
+        try:
+            ShardedBucket(plan, local=local)
+            msg = "no error"
+        except RuntimeError as e:
+            msg = str(e)
+        with open(os.path.join(outdir, f"rank{rank}.txt"), "w") as f:
+            f.write(msg)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_ranks_that_disagree_on_the_plan_all_fail_at_construction(tmp_path):
+    world = 2
+    mp.start_processes(_disagree_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    for r in range(world):
+        msg = (tmp_path / f"rank{r}.txt").read_text()
+        assert "disagree on the bucket plan" in msg and "[1]" in msg, msg
