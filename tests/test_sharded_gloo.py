@@ -15,6 +15,7 @@ over up to four ranks is exact in bf16 whatever order the reduction takes.
 import datetime
 import os
 import socket
+import time
 
 import numpy as np
 import pytest
@@ -410,3 +411,38 @@ def test_ranks_that_disagree_on_the_plan_all_fail_at_construction(tmp_path):
     for r in range(world):
         msg = (tmp_path / f"rank{r}.txt").read_text()
         assert "disagree on the bucket plan" in msg and "[1]" in msg, msg
+
+
+def _leaver_worker(rank, world, port, outdir):
+    """Rank 1 leaves between steps (after one step, with nothing in flight);
+    rank 0's next step must end with an error, not wait for ever."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=10))
+    import oracle
+    import ragged_bucket_layout_b200 as rb
+    from ragged_bucket_layout_b200.sharded import ShardedBucket
+
+    rows, cols, k, bc = CASES["tiny"]
+    plan = rb.dbuf_plan(rows, cols, k, world, 16, block_cols=bc)
+    info = rb.dbuf_plan_info(plan)
+    local = OracleSlice(oracle.rank_bucket(rows, cols, k, info["offsets"], info["slice"], world, rank, bc))
+    sb = ShardedBucket(plan, local=local)
+    sb.step(_hp(1))
+    if rank == 1:
+        return                                   # leaves: its sockets close when the process exits
+    t0 = time.monotonic()
+    try:
+        sb.step(_hp(2))
+        msg = "no error"
+    except RuntimeError as e:
+        msg = f"error after {time.monotonic() - t0:.1f} s: {type(e).__name__}"
+    with open(os.path.join(outdir, "rank0.txt"), "w") as f:
+        f.write(msg)
+
+
+def test_a_rank_that_leaves_makes_the_next_step_fail(tmp_path):
+    mp.start_processes(_leaver_worker, args=(2, _free_port(), str(tmp_path)), nprocs=2, join=True,
+                       start_method="spawn")
+    msg = (tmp_path / "rank0.txt").read_text()
+    assert msg.startswith("error after"), msg
+    assert float(msg.split()[2]) < 30.0, msg
