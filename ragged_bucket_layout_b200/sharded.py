@@ -33,8 +33,10 @@ class ShardedBucket:
     """Rank `rank` of `world` for the bucket of `plan` (planned with
     m = world).  `local` replaces the slice bucket (a DBuffer of
     dbuf_plan_rank(plan, rank) on `device` by default) with any object that
-    has array(which), views(which) and step(hp, grad_scale), e.g. a host-side
-    model of it."""
+    has array(which), views(which) and step(hp, grad_scale), plus
+    grad_norm(grad_scale, out) for step_clipped, e.g. a host-side model of
+    it.  With NCCL, make the rank's GPU the current device first (the plan
+    check and the collectives run there)."""
 
     def __init__(self, plan, rank=None, world=None, group=None, device="cuda", local=None, check_plan=True):
         """check_plan: compare a digest of the plan across the group first
