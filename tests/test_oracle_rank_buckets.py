@@ -8,7 +8,9 @@ itself:
     bit (master, bf16 copy, codes, scales);
   * its first block is the number of whole-bucket blocks that start before
     the slice (oracle.tiles numbering);
-  * the parts of every tensor follow one another rank by rank and cover it.
+  * the parts of every tensor follow one another rank by rank and cover it;
+  * they are the RaggedShard rows of oracle.shards, and their padding laid
+    side by side is the whole bucket's.
 """
 import numpy as np
 import pytest
@@ -138,3 +140,20 @@ def test_a_cut_block_is_refused():
     elements (3 rows) has its first block cut."""
     with pytest.raises(AssertionError):
         oracle.rank_bucket([8], [16], [4], [0], 48, 3, 1)
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_rank_buckets_agree_with_the_shard_rows_and_the_padding(name):
+    """Two other oracle functions, written separately, say the same: the
+    RaggedShard rows of each rank (oracle.shards) are the rank buckets'
+    parts, and the rank buckets' padding laid side by side is the whole
+    bucket's padding."""
+    r, c, k, bc, m, off, s = _layout(name)
+    rows_of = oracle.shards(r, c, off, s, m)
+    pad = []
+    for q in range(m):
+        rk = oracle.rank_bucket(r, c, k, off, s, m, q, bc)
+        want = [(i, a, b) for i, per in enumerate(rows_of) for a, b in [per[q]] if b > a]
+        assert rk["parts"] == want
+        pad.append(oracle.padding_mask(rk["rows"], rk["cols"], rk["offsets"], s))
+    assert np.array_equal(np.concatenate(pad), oracle.padding_mask(r, c, off, m * s))
