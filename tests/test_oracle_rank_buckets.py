@@ -10,7 +10,9 @@ itself:
     the slice (oracle.tiles numbering);
   * the parts of every tensor follow one another rank by rank and cover it;
   * they are the RaggedShard rows of oracle.shards, and their padding laid
-    side by side is the whole bucket's.
+    side by side is the whole bucket's;
+  * on the tiny layout they equal the hand-worked values in
+    tests/golden/rank_buckets_tiny.json.
 """
 import numpy as np
 import pytest
@@ -157,3 +159,18 @@ def test_rank_buckets_agree_with_the_shard_rows_and_the_padding(name):
         assert rk["parts"] == want
         pad.append(oracle.padding_mask(rk["rows"], rk["cols"], rk["offsets"], s))
     assert np.array_equal(np.concatenate(pad), oracle.padding_mask(r, c, off, m * s))
+
+
+def test_golden_rank_buckets_of_the_tiny_layout(golden_dir):
+    """The rank buckets of the tiny layout, worked by hand
+    (tests/golden/rank_buckets_tiny.json)."""
+    import json
+    import os
+    g = json.load(open(os.path.join(golden_dir, "rank_buckets_tiny.json")))
+    for q, want in enumerate(g["ranks"]):
+        rk = oracle.rank_bucket(g["rows"], g["cols"], g["k"], g["offsets"], g["s"], g["m"], q)
+        assert [list(p) for p in rk["parts"]] == want["parts"]
+        assert rk["offsets"].tolist() == want["offsets"]
+        assert rk["first_block"] == want["first_block"]
+        assert int(oracle.padding_mask(rk["rows"], rk["cols"], rk["offsets"], g["s"]).sum()) == want["padding"]
+        assert oracle.blocks(rk["rows"], rk["cols"], rk["k"], rk["offsets"])[0].size == want["n_blocks"]

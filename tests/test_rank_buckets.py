@@ -114,3 +114,19 @@ def test_rank_parts_agree_with_the_shard_table(name):
         assert rb.dbuf_plan_dims(R) == (len(R.parts), 1)
         want = [int(off[i]) + a * int(c[i]) - q * s for i, a, b in R.parts]
         assert rb.dbuf_plan_info(R)["offsets"] == want
+
+
+def test_golden_rank_buckets_of_the_tiny_layout(golden_dir):
+    """The library's rank plans of the tiny layout against the hand-worked
+    values in tests/golden/rank_buckets_tiny.json."""
+    import json
+    import os
+    g = json.load(open(os.path.join(golden_dir, "rank_buckets_tiny.json")))
+    P = rb.dbuf_plan(g["rows"], g["cols"], g["k"], g["m"], 16)
+    assert rb.dbuf_plan_info(P)["offsets"] == g["offsets"] and rb.dbuf_plan_info(P)["slice"] == g["s"]
+    for q, want in enumerate(g["ranks"]):
+        R = rb.dbuf_plan_rank(P, q)
+        info = rb.dbuf_plan_info(R)
+        assert [list(p) for p in R.parts] == want["parts"]
+        assert info["offsets"] == want["offsets"] and info["padding"] == want["padding"]
+        assert info["n_blocks"] == want["n_blocks"] and R.first_block == want["first_block"]
