@@ -174,3 +174,44 @@ def test_golden_rank_buckets_of_the_tiny_layout(golden_dir):
         assert rk["first_block"] == want["first_block"]
         assert int(oracle.padding_mask(rk["rows"], rk["cols"], rk["offsets"], g["s"]).sum()) == want["padding"]
         assert oracle.blocks(rk["rows"], rk["cols"], rk["k"], rk["offsets"])[0].size == want["n_blocks"]
+
+
+def test_random_buckets_step_like_the_whole_bucket():
+    """60 seeded random buckets (ragged rows and blocks, some 2-D blocks, m up
+    to 6), two steps: every rank bucket stepped alone equals its slice of
+    the whole bucket."""
+    rng = np.random.default_rng(77)
+    for case in range(60):
+        n = int(rng.integers(1, 6))
+        r, c, k, bc = [], [], [], []
+        for _ in range(n):
+            tiled = rng.random() < 0.3
+            C = int(rng.choice([16, 32, 48])) if tiled else int(rng.integers(1, 50))
+            R = int(rng.integers(1, 60))
+            r.append(R)
+            c.append(C)
+            k.append(int(rng.integers(1, R + 1)))
+            bc.append(16 if tiled and C > 16 else 0)
+        m = int(rng.integers(1, 7))
+        st, off, s = oracle.plan(r, c, k, m, 16)
+        assert st == oracle.OK
+        W = oracle.Bucket(r, c, k, off, s, m, block_cols=bc)
+        _fill_params(W, r, c, off, case)
+        ranks = [oracle.rank_bucket(r, c, k, off, s, m, q, bc) for q in range(m)]
+        B = [oracle.Bucket(x["rows"], x["cols"], x["k"], x["offsets"], s, 1, block_cols=x["block_cols"])
+             for x in ranks]
+        for q in range(m):
+            B[q].p[:] = W.p[q * s:(q + 1) * s]
+        for t in (1, 2):
+            hp = dict(synth.HPARAMS, step=t)
+            W.g[:] = _grads(r, c, off, W.size, case, t)
+            W.step(hp, t, 1.0 / m)
+            for q in range(m):
+                B[q].g[:] = W.g[q * s:(q + 1) * s]
+                B[q].step(hp, t, 1.0 / m)
+        for q in range(m):
+            sl = slice(q * s, (q + 1) * s)
+            assert np.array_equal(B[q].p.view(np.uint32), W.p[sl].view(np.uint32)), (case, q)
+            assert np.array_equal(B[q].pb, W.pb[sl]) and np.array_equal(B[q].mq, W.mq[sl]), (case, q)
+            fb = ranks[q]["first_block"]
+            assert np.array_equal(B[q].scale_v, W.scale_v[fb:fb + B[q].scale_v.size]), (case, q)

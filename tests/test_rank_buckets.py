@@ -130,3 +130,44 @@ def test_golden_rank_buckets_of_the_tiny_layout(golden_dir):
         assert [list(p) for p in R.parts] == want["parts"]
         assert info["offsets"] == want["offsets"] and info["padding"] == want["padding"]
         assert info["n_blocks"] == want["n_blocks"] and R.first_block == want["first_block"]
+
+
+def _random_bucket(rng):
+    n = int(rng.integers(1, 8))
+    rows, cols, k, bc = [], [], [], []
+    for _ in range(n):
+        tiled = rng.random() < 0.3
+        C = int(rng.choice([16, 32, 48, 64])) if tiled else int(rng.integers(1, 70))
+        R = int(rng.integers(1, 90))
+        rows.append(R)
+        cols.append(C)
+        k.append(int(rng.integers(1, R + 1)))
+        bc.append(int(rng.choice([16, 32])) if tiled and C > 16 else 0)
+    return rows, cols, k, bc, int(rng.integers(1, 9))
+
+
+def test_random_buckets_rank_plans_and_work_tables():
+    """300 seeded random buckets (1-7 tensors, ragged rows and blocks, some
+    2-D blocks, m up to 8): for every rank the library's rank plan equals
+    the oracle's rank bucket and its work table is the parent's slice."""
+    rng = np.random.default_rng(2024)
+    for _ in range(300):
+        rows, cols, k, bc, m = _random_bucket(rng)
+        P = rb.dbuf_plan(rows, cols, k, m, 16, block_cols=bc)
+        info = rb.dbuf_plan_info(P)
+        s, off = info["slice"], info["offsets"]
+        parent = rb.dbuf_work_table(P)
+        for q in range(m):
+            R = rb.dbuf_plan_rank(P, q)
+            want = oracle.rank_bucket(rows, cols, k, off, s, m, q, bc)
+            ri = rb.dbuf_plan_info(R)
+            assert R.parts == want["parts"] and ri["offsets"] == want["offsets"].tolist()
+            assert R.first_block == want["first_block"]
+            exp = []
+            for e in parent:
+                if q * s <= e["first_elem"] < (q + 1) * s:
+                    x = dict(e, first_elem=e["first_elem"] - q * s)
+                    if e["kind"] != 2:
+                        x["first_block"] = e["first_block"] - R.first_block
+                    exp.append(x)
+            assert rb.dbuf_work_table(R) == exp, (rows, cols, k, bc, m, q)
