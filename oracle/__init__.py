@@ -5,7 +5,8 @@ Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 library.  The planner and the 8-bit Adam step live in ``oracle.cpp`` (plain
 C++, fp32 in one fixed operation order); this module marshals numpy arrays
 for them and holds, in plain numpy, the row-wise (FSDP2-style) baseline
-layout and the Muon pieces (fp32 momentum, float64 Newton-Schulz).
+layout, the rank buckets (one device's slice as a bucket of its own) and
+the Muon pieces (fp32 momentum, float64 Newton-Schulz).
 
 Every function cites the part of the veScale-FSDP description it follows; the
 parity status of each is stated in ``oracle.cpp``'s header.
