@@ -91,3 +91,20 @@ def test_algorithmic_bytes_of_the_tiny_and_llama_buckets():
         st = bench.workload_stats(w, info)
         assert (st["params"], st["blocks"], st["padding"], st["step_bytes"]) == (P, B, pad, total)
         assert st["copy_in_bytes"] == 4 * P
+
+
+def test_reference_arm_on_other_ranks_exits_without_work():
+    """Under torchrun with N > 1 only rank 0 runs and prints the reference
+    arm; another rank exits 0 at once and prints no JSON line."""
+    import subprocess
+    import sys
+    import time
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, RANK="1", LOCAL_RANK="1", WORLD_SIZE="2")
+    t0 = time.monotonic()
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--gpus", "2",
+                          "--steps", "1", "--warmup", "1"], capture_output=True, text=True, timeout=300, cwd=root,
+                         env=env)
+    assert out.returncode == 0, out.stderr[-2000:]
+    assert not [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert time.monotonic() - t0 < 120
