@@ -62,6 +62,9 @@ def workload_stats(w, info):
                 step_bytes=16 * P + 16 * B + 2 * pad, copy_in_bytes=4 * P)
 
 
+NOMINAL_HBM_GBS = 8000.0   # B200 nominal HBM3e bandwidth (8 TB/s, the DGX figure)
+
+
 def measured_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -529,6 +532,7 @@ def run_ours(args):
     peak, peak_src = measured_peak()
     roof = {"bound": "hbm", "achieved": kernel_gbs, "peak": peak, "unit": "GB/s", "frac": kernel_gbs / peak,
             "traffic": profiled_traffic(w.name, stats), "peak_source": peak_src,
+            "frac_of_nominal_8tbs": kernel_gbs / NOMINAL_HBM_GBS,
             "kernel": "adam8_step_kernel", "algorithmic_bytes_per_launch": stats["step_bytes"]}
 
     cpu = None
