@@ -131,7 +131,8 @@ dbuf_status dbuf_plan_shards(const dbuf_plan_t* plan, dbuf_shard_rows* out);
  * bit for bit. It stores the fp32 master weights, codes and scales of that
  * one slice only.  *first_block (may be NULL) receives the parent's index of
  * its block 0.  rank in [0, m); *out (freed with dbuf_plan_free) is NULL on
- * failure.  Host only. */
+ * failure.  DBUF_EINVAL for a rank out of range, or if a slice boundary cuts
+ * a block (which no plan from dbuf_plan does).  Host only. */
 dbuf_status dbuf_plan_rank(const dbuf_plan_t* plan, int32_t rank, dbuf_plan_t** out, int64_t* first_block);
 
 /* Bytes of device memory dbuf_create needs for this plan (one allocation:
